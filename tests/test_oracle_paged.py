@@ -1,0 +1,75 @@
+"""Pins for the oracle's paged-cache indexing (append scatter, gather)."""
+
+import numpy as np
+
+from oracle import e4m3, paged
+
+
+def _pattern_pages(P, Hkv, ps, D):
+    # every byte names its own coordinates, so a wrong index is visible
+    p, h, s, d = np.meshgrid(np.arange(P), np.arange(Hkv), np.arange(ps), np.arange(D),
+                             indexing="ij")
+    return ((p * 7 + h * 31 + s * 5 + d * 3) % 251).astype(np.uint8)
+
+
+def test_gather_codes_follows_block_table_slot_by_slot():
+    P, Hkv, ps, D = 9, 3, 4, 5
+    pages = _pattern_pages(P, Hkv, ps, D)
+    table = np.array([[7, 2, 5, -1], [0, 8, -1, -1]], dtype=np.int32)
+    for b, L in [(0, 11), (1, 5), (0, 1), (1, 8)]:
+        got = paged.gather_codes(pages, table, b, L, ps)
+        assert got.shape == (L, Hkv, D)
+        for t in range(L):
+            page = table[b][t // ps]
+            for h in range(Hkv):
+                assert np.array_equal(got[t, h], pages[page, h, t % ps])
+
+
+def test_gather_dequant_applies_the_head_scale():
+    P, Hkv, ps, D = 4, 2, 4, 3
+    pages = np.full((P, Hkv, ps, D), 0x38, np.uint8)        # 1.0 everywhere
+    table = np.array([[3, 1]], dtype=np.int32)
+    scale = np.array([0.5, 3.0], np.float32)
+    x = paged.gather_dequant(pages, scale, table, 0, 6, ps)
+    assert np.array_equal(x[:, 0], np.full((6, D), 0.5))
+    assert np.array_equal(x[:, 1], np.full((6, D), 3.0))
+
+
+def test_append_writes_exactly_the_new_slots():
+    rng = np.random.default_rng(5)
+    P, Hkv, ps, D = 12, 2, 4, 8
+    pages = rng.integers(0, 256, (P, Hkv, ps, D), dtype=np.uint8)
+    table = np.array([[4, 9, 1, -1], [0, 11, 6, 3]], dtype=np.int32)
+    start = np.array([3, 6], np.int32)
+    n_new = 5
+    new = rng.standard_normal((2, n_new, Hkv, D)).astype(np.float32)
+    scale = np.array([0.02, 0.3], np.float32)
+    out = paged.append(pages, new, scale, table, start, ps)
+    touched = np.zeros(pages.shape, bool)
+    for b in range(2):
+        for t in range(n_new):
+            pos = start[b] + t
+            page, slot = table[b][pos // ps], pos % ps
+            for h in range(Hkv):
+                want = e4m3.encode(new[b, t, h], scale[h])
+                assert np.array_equal(out[page, h, slot], want)
+                touched[page, h, slot] = True
+    assert np.array_equal(out[~touched], pages[~touched])
+    assert np.array_equal(pages, np.asarray(pages))                  # input untouched
+
+
+def test_append_in_two_calls_equals_one_call():
+    rng = np.random.default_rng(6)
+    P, Hkv, ps, D = 8, 1, 4, 4
+    pages = np.zeros((P, Hkv, ps, D), np.uint8)
+    table = np.array([[5, 2, 7]], dtype=np.int32)
+    new = rng.standard_normal((1, 10, Hkv, D)).astype(np.float32)
+    scale = np.array([0.01], np.float32)
+    one = paged.append(pages, new, scale, table, np.array([0]), ps)
+    two = paged.append(pages, new[:, :3], scale, table, np.array([0]), ps)
+    two = paged.append(two, new[:, 3:], scale, table, np.array([3]), ps)
+    assert np.array_equal(one, two)
+    back = paged.gather_dequant(one, scale, table, 0, 10, ps)
+    # the round trip is within half an E4M3 step (relative 1/16) of the input
+    err = np.abs(back[:, 0] - new[0, :, 0])
+    assert np.all(err <= np.abs(new[0, :, 0]) / 16 + 2.0 ** -10 * scale[0])
