@@ -1,0 +1,204 @@
+/*
+ * atlas_kv.h -- C ABI of the paged FP8 KV-cache decode / MTP-verify attention
+ * library for NVIDIA B200 (sm_100a).  Library: libatlas_kv.so.
+ *
+ * What the library computes.  The Atlas pages describe an inference engine
+ * with a "paged FP8 KV cache" and multi-token-prediction (MTP, K = 4 drafts)
+ * verification (GB10 page: "Atlas Takes On vLLM With a Pure Rust/CUDA
+ * Inference Engine on a Single GB10", deployment-path paragraph), a memory
+ * pool of fixed-size preallocated blocks for the KV cache (Atlas deep-dive,
+ * ainews.cool, "Memory architecture" paragraph), FP8 quantisation with scale
+ * factors (same page, "Quantisation" paragraph) and dedicated MQA/GQA
+ * attention kernels of the FlashAttention-2 family (same page, "Attention"
+ * paragraph).  The pages fix no layout, page size, scale granularity,
+ * rounding or mask convention; the readings used here are:
+ *
+ *   pages        uint8 E4M3 codes, layout [num_pages][num_kv_heads][page_size][head_dim]
+ *   block table  int32 [batch][max_blocks_per_seq]; token p of sequence b is in
+ *                page block_table[b][p / page_size], slot p % page_size
+ *   scales       one float32 per KV head for K and one for V (static)
+ *   encode       code = E4M3(fp32(x) / fp32(scale[h])), IEEE division, round to
+ *                nearest even, |y| >= 448 saturates to +-448, sign of zero kept
+ *   q, out       bf16 [batch][q_len][num_q_heads][head_dim]; q-head hq reads KV
+ *                head hq / (num_q_heads / num_kv_heads)
+ *   seq_lens     context length of each sequence INCLUDING the q_len new tokens,
+ *                whose K/V must already be appended
+ *   mask         new row i (0-based) sees key positions t <= seq_len - q_len + i
+ *   softmax      s = sm_scale * q . k, fp32 online softmax, fp32 accumulation,
+ *                bf16 output (round to nearest even); sm_scale <= 0 means
+ *                1/sqrt(head_dim)
+ *
+ * Ownership.  Every buffer is owned by the caller; the library stores
+ * pointers and never allocates or frees device memory.  A pool handle is
+ * owned by the caller from atlas_kv_pool_create until atlas_kv_pool_destroy.
+ *
+ * Streams.  Every compute entry point only enqueues work on the given stream
+ * (a cudaStream_t passed as void*; NULL = legacy default stream) and returns
+ * without synchronising.  Only atlas_get_device_error synchronises.
+ *
+ * Errors.  Arguments are checked on the host before anything is enqueued;
+ * a failed check returns a negative status and enqueues nothing.  Checks
+ * that need device data (page ids inside the block table, per-sequence
+ * lengths, append positions) are made by the kernels: an offending page or
+ * sequence is skipped (its output rows are written as zeros or left
+ * untouched, as documented per call) and a bit is set in the pool's device
+ * error word, read with atlas_get_device_error.  No kernel traps.
+ *
+ * Threads.  A pool is immutable after creation except for its workspace.
+ * Decode calls that share one pool share its workspace, so they must be
+ * issued on one stream (or otherwise ordered); appends do not use the
+ * workspace.
+ */
+#ifndef ATLAS_KV_H
+#define ATLAS_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATLAS_API __attribute__((visibility("default")))
+#else
+#define ATLAS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct atlas_kv_pool atlas_kv_pool_t;   /* opaque host-side descriptor */
+
+typedef enum {
+    ATLAS_OK = 0,
+    ATLAS_ERR_INVALID_ARG = -1,   /* null pointer, bad size or alignment        */
+    ATLAS_ERR_UNSUPPORTED = -2,   /* a shape this build has no kernel for       */
+    ATLAS_ERR_WORKSPACE = -3,     /* workspace too small for the call           */
+    ATLAS_ERR_CUDA = -4,          /* a CUDA runtime call failed                 */
+    ATLAS_ERR_DEVICE_CHECK = -5   /* atlas_get_device_error found a device flag */
+} atlas_status_t;
+
+typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
+
+/* Bits of the device error word. */
+#define ATLAS_DEVERR_PAGE_ID   0x1   /* decode: block-table entry outside [0, num_pages) */
+#define ATLAS_DEVERR_SEQ_LEN   0x2   /* decode: seq_len < q_len, > max_seq_len or > table */
+#define ATLAS_DEVERR_APPEND    0x4   /* append: position or page id out of range          */
+
+/* Fields of atlas_paged_gqa_decode_plan's output array. */
+#define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split                           */
+#define ATLAS_PLAN_NUM_SPLITS    1   /* splits for max_seq_len                        */
+#define ATLAS_PLAN_KERNEL        2   /* 1 = warp-level mma.sync kernel                */
+#define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) handled per CTA    */
+#define ATLAS_PLAN_ROW_BLOCKS    4   /* CTAs per (split, KV head, sequence)           */
+#define ATLAS_PLAN_LAUNCHES      5   /* kernel launches per decode call               */
+#define ATLAS_PLAN_GRID_CTAS     6   /* CTAs launched (empty splits exit at once)     */
+#define ATLAS_PLAN_FIELDS        7
+
+/*
+ * Bytes of workspace a pool needs so that decode calls with batch <=
+ * max_batch, q_len <= max_q_len, the given num_q_heads and head_dim and
+ * max_seq_len <= max_seq_len fit, for any split size >= min_split_tokens
+ * (<= 0 selects 64, the smallest split the library uses on its own).
+ * The workspace holds the split-KV partial results (float32 O rows and
+ * log-sum-exp values), one completion counter per (sequence, KV head, row
+ * block) and the device error word.  Returns 0 for invalid arguments.
+ */
+ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t num_q_heads,
+                                int32_t head_dim, int32_t max_seq_len,
+                                int32_t min_split_tokens);
+
+/*
+ * Describe a page pool.  num_pages >= 1; page_size a multiple of 16 and
+ * <= 1024; head_dim 64 or 128; num_kv_heads >= 1.  k_pages / v_pages: device
+ * uint8 [num_pages][num_kv_heads][page_size][head_dim], 16-byte aligned.
+ * k_scale / v_scale: device float32 [num_kv_heads] (used by append; decode
+ * takes its own scale pointers).  max_batch, max_q_len, num_q_heads bound the
+ * decode calls (they size the counter region).  workspace: device memory of
+ * workspace_bytes >= atlas_kv_workspace_bytes(...), 256-byte aligned and
+ * ZERO-FILLED by the caller before the first call; the library keeps its
+ * counters at zero between calls.  No CUDA call is made here.
+ */
+ATLAS_API atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** pool, int32_t num_pages,
+                                    int32_t page_size, int32_t num_kv_heads,
+                                    int32_t head_dim, void* k_pages, void* v_pages,
+                                    const float* k_scale, const float* v_scale,
+                                    int32_t max_batch, int32_t max_q_len,
+                                    int32_t num_q_heads, void* workspace,
+                                    size_t workspace_bytes);
+
+/* Free the host-side descriptor (not the caller's buffers).  NULL is a no-op. */
+ATLAS_API atlas_status_t atlas_kv_pool_destroy(atlas_kv_pool_t* pool);
+
+/*
+ * Override the KV split size (tokens per split) of later decode calls; 0
+ * restores the automatic choice.  Must be 0 or a multiple of 64 in
+ * [64, 8192].  Meant for tuning and for split-invariance tests.
+ */
+ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, int32_t split_tokens);
+
+/*
+ * FP8 page append (quantise + scatter), the cache-fill step.
+ * k_new / v_new: device [batch][n_new][num_kv_heads][head_dim] of dtype
+ * (float32 or bf16), 16-byte aligned.  block_table: device int32
+ * [batch][max_blocks_per_seq].  start_pos: device int32 [batch], position of
+ * the first new token of each sequence.  Token t of sequence b is written to
+ * position start_pos[b] + t with code E4M3(fp32(x) / fp32(scale[h])) using the
+ * pool's k_scale / v_scale; the result is bit-exact with that definition.
+ * Rows whose position is negative, past max_blocks_per_seq*page_size, or
+ * whose page id is outside [0, num_pages) are skipped and flag
+ * ATLAS_DEVERR_APPEND.  batch == 0 or n_new == 0 is a no-op.
+ */
+ATLAS_API atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_new,
+                                   const void* v_new, int32_t dtype,
+                                   const int32_t* block_table, int32_t max_blocks_per_seq,
+                                   const int32_t* start_pos, int32_t batch, int32_t n_new,
+                                   void* stream);
+
+/*
+ * Paged decode (q_len == 1) / MTP-verify (q_len > 1) grouped-query attention.
+ * q: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
+ * k_pages / v_pages: the pool's page arrays (or arrays of identical shape).
+ * k_scale / v_scale: device float32 [num_kv_heads].  block_table: device
+ * int32 [batch][max_blocks_per_seq]; only the first ceil(seq_len/page_size)
+ * entries of a row are read.  seq_lens: device int32 [batch].
+ * max_seq_len: host upper bound of seq_lens (sizes the split grid).
+ * out: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
+ * A sequence with seq_len < q_len, seq_len > max_blocks_per_seq*page_size or
+ * seq_len > max_seq_len gets zero output rows and flags ATLAS_DEVERR_SEQ_LEN; a page id outside
+ * [0, num_pages) is skipped (its tokens do not take part) and flags
+ * ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
+                                      const void* k_pages, const void* v_pages,
+                                      const float* k_scale, const float* v_scale,
+                                      const int32_t* block_table,
+                                      int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                      int32_t batch, int32_t num_q_heads, int32_t q_len,
+                                      int32_t max_seq_len, float sm_scale, void* out,
+                                      void* stream);
+
+/*
+ * The launch plan a decode call with these arguments would use (host only,
+ * no CUDA call).  Writes min(n, ATLAS_PLAN_FIELDS) int32 fields to plan.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t batch,
+                                           int32_t num_q_heads, int32_t q_len,
+                                           int32_t max_seq_len, int32_t* plan, int32_t n);
+
+/*
+ * Wait for the stream, read the pool's device error word into *code and
+ * clear it.  Returns ATLAS_OK if it was zero, ATLAS_ERR_DEVICE_CHECK if not.
+ */
+ATLAS_API atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream,
+                                      int32_t* code);
+
+/* Static description of a status code. */
+ATLAS_API const char* atlas_status_string(atlas_status_t status);
+
+/* Library version, e.g. "0.1.0". */
+ATLAS_API const char* atlas_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATLAS_KV_H */

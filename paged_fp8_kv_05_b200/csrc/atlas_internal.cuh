@@ -1,0 +1,120 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+// Device helpers here wrap single PTX instructions (conversion, warp MMA,
+// register-matrix transpose, base-2 exponential); none re-implements a
+// math-library routine.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "atlas_kv.h"
+
+namespace atlas {
+
+// ---------------------------------------------------------------- parameters
+
+struct AppendParams {
+  const void* k_new;          // [B][n_new][Hkv][D] f32 or bf16
+  const void* v_new;
+  int dtype;                  // ATLAS_DTYPE_*
+  uint8_t* k_pages;           // [P][Hkv][ps][D]
+  uint8_t* v_pages;
+  const float* k_scale;       // [Hkv]
+  const float* v_scale;
+  const int32_t* block_table; // [B][max_blocks]
+  const int32_t* start_pos;   // [B]
+  int32_t* err;               // device error word
+  int batch, n_new, Hkv, D, ps, num_pages, max_blocks;
+};
+
+struct DecodeParams {
+  const __nv_bfloat16* q;     // [B][q_len][Hq][D]
+  const uint8_t* k_pages;     // [P][Hkv][ps][D]
+  const uint8_t* v_pages;
+  const float* k_scale;       // [Hkv]
+  const float* v_scale;
+  const int32_t* block_table; // [B][max_blocks]
+  const int32_t* seq_lens;    // [B]
+  __nv_bfloat16* out;         // [B][q_len][Hq][D]
+  float* part_o;              // [B][num_splits][q_len*Hq][D]   (split partials)
+  float* part_lse;            // [B][num_splits][q_len*Hq]       (log2-domain LSE)
+  int32_t* counters;          // [B][Hkv][row_blocks], zero between calls
+  int32_t* err;               // device error word
+  int B, Hq, Hkv, G, q_len, D, ps, num_pages, max_blocks;
+  int split_tokens, num_splits, row_blocks;
+  float qk_scale_log2;        // sm_scale * log2(e); k_scale[h] is folded in per head
+};
+
+cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
+
+// rows_per_cta is 8 or 16; grid = (num_splits * row_blocks, Hkv, B)
+cudaError_t launch_decode_mma(const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
+size_t decode_mma_smem_bytes(int D, int rows_per_cta, int split_tokens);
+
+// ------------------------------------------------------------ device helpers
+
+#ifdef __CUDACC__
+
+// Two E4M3 codes (low byte first) -> f16x2 (exact: E4M3 is a subset of f16).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// f16x2 with `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// D += A * B, m16n8k16, f16 inputs, f32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one b32 pair per thread.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+// Hardware base-2 exponential (ex2.approx); ex2(-inf) = +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Streaming 16-byte / 8-byte read-only loads that skip L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint2 ld_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+#endif  // __CUDACC__
+
+}  // namespace atlas

@@ -1,0 +1,328 @@
+// C-ABI layer of libatlas_kv.so: argument checks, launch planning and the
+// entry points declared in include/atlas_kv.h.  Owns no device memory.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "atlas_internal.cuh"
+
+struct atlas_kv_pool {
+  int32_t num_pages, page_size, num_kv_heads, head_dim;
+  uint8_t* k_pages;
+  uint8_t* v_pages;
+  const float* k_scale;
+  const float* v_scale;
+  int32_t max_batch, max_q_len, num_q_heads;
+  uint8_t* workspace;
+  size_t workspace_bytes;
+  int32_t split_override;
+  // workspace layout, fixed at creation
+  size_t counters_off, counters_slots, partial_off;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kDefaultSms = 148;          // B200; used only when no device is visible
+constexpr int kMinSplit = 64;             // 4 warps x 16-token units
+constexpr int kMaxSplit = 8192;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return kDefaultSms;
+  }
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return kDefaultSms;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+size_t partial_bytes(int batch, int num_splits, int rows_all, int head_dim) {
+  const size_t lse = align_up((size_t)batch * num_splits * rows_all * sizeof(float), kAlign);
+  const size_t o = align_up((size_t)batch * num_splits * rows_all * head_dim * sizeof(float), kAlign);
+  return lse + o;
+}
+
+struct Plan {
+  int split_tokens, num_splits, kernel, rows_per_cta, row_blocks, launches;
+  long long grid_ctas;
+};
+
+// Split-KV partition (A1).  The host sees only max_seq_len, so it sizes the
+// grid as if every sequence were that long; splits past a sequence's end exit
+// at once.  Target about two waves of 4 resident CTAs per SM, splits a multiple
+// of 64 tokens in [kMinSplit, kMaxSplit]; the chunk adapts to the sequence
+// length and the SM count, the "block size adapted to sequence length and
+// architecture" of the Atlas deep-dive's attention paragraph.
+Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len, int max_seq_len,
+               int sms) {
+  Plan pl;
+  const int G = num_q_heads / pool->num_kv_heads;
+  const int R = q_len * G;
+  pl.kernel = 1;
+  pl.rows_per_cta = (R <= 8) ? 8 : 16;
+  pl.row_blocks = (R + pl.rows_per_cta - 1) / pl.rows_per_cta;
+  int T;
+  if (pool->split_override > 0) {
+    T = pool->split_override;
+  } else {
+    const long long units = (long long)batch * pool->num_kv_heads * pl.row_blocks;
+    const long long target = (long long)sms * 4 * 2;
+    long long want = (target + units - 1) / (units > 0 ? units : 1);
+    if (want < 1) want = 1;
+    long long t = (max_seq_len + want - 1) / want;
+    t = (t + kMinSplit - 1) / kMinSplit * kMinSplit;
+    if (t < 256) t = 256;
+    if (t > kMaxSplit) t = kMaxSplit;
+    T = (int)t;
+  }
+  pl.split_tokens = T;
+  pl.num_splits = (max_seq_len + T - 1) / T;
+  if (pl.num_splits < 1) pl.num_splits = 1;
+  pl.launches = 1;
+  pl.grid_ctas = (long long)pl.num_splits * pl.row_blocks * pool->num_kv_heads * batch;
+  return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* atlas_version(void) { return "0.1.0"; }
+
+const char* atlas_status_string(atlas_status_t s) {
+  switch (s) {
+    case ATLAS_OK: return "ok";
+    case ATLAS_ERR_INVALID_ARG: return "invalid argument";
+    case ATLAS_ERR_UNSUPPORTED: return "unsupported shape";
+    case ATLAS_ERR_WORKSPACE: return "workspace too small";
+    case ATLAS_ERR_CUDA: return "CUDA runtime error";
+    case ATLAS_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t num_q_heads,
+                                int32_t head_dim, int32_t max_seq_len, int32_t min_split_tokens) {
+  if (max_batch < 0 || max_q_len < 1 || num_q_heads < 1 || max_seq_len < 0) return 0;
+  if (head_dim != 64 && head_dim != 128) return 0;
+  if (min_split_tokens <= 0) min_split_tokens = kMinSplit;
+  const int max_splits = (max_seq_len + min_split_tokens - 1) / min_split_tokens;
+  const size_t counters = align_up((size_t)max_batch * num_q_heads * max_q_len * sizeof(int32_t), kAlign);
+  return kAlign + counters +
+         partial_bytes(max_batch, max_splits > 0 ? max_splits : 1, max_q_len * num_q_heads, head_dim);
+}
+
+atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, int32_t page_size,
+                                    int32_t num_kv_heads, int32_t head_dim, void* k_pages,
+                                    void* v_pages, const float* k_scale, const float* v_scale,
+                                    int32_t max_batch, int32_t max_q_len, int32_t num_q_heads,
+                                    void* workspace, size_t workspace_bytes) {
+  if (!out) return ATLAS_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (num_pages < 1 || num_kv_heads < 1 || max_batch < 0 || max_q_len < 1 || num_q_heads < 1)
+    return ATLAS_ERR_INVALID_ARG;
+  if (page_size < 16 || page_size > 1024 || page_size % 16 != 0) return ATLAS_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return ATLAS_ERR_INVALID_ARG;
+  if (!k_pages || !v_pages || !k_scale || !v_scale || !workspace) return ATLAS_ERR_INVALID_ARG;
+  if (!aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(workspace, kAlign))
+    return ATLAS_ERR_INVALID_ARG;
+  const size_t counters_slots = (size_t)max_batch * num_q_heads * max_q_len;
+  const size_t counters_bytes = align_up(counters_slots * sizeof(int32_t), kAlign);
+  if (workspace_bytes < kAlign + counters_bytes) return ATLAS_ERR_WORKSPACE;
+  atlas_kv_pool* p = new (std::nothrow) atlas_kv_pool;
+  if (!p) return ATLAS_ERR_INVALID_ARG;
+  p->num_pages = num_pages;
+  p->page_size = page_size;
+  p->num_kv_heads = num_kv_heads;
+  p->head_dim = head_dim;
+  p->k_pages = static_cast<uint8_t*>(k_pages);
+  p->v_pages = static_cast<uint8_t*>(v_pages);
+  p->k_scale = k_scale;
+  p->v_scale = v_scale;
+  p->max_batch = max_batch;
+  p->max_q_len = max_q_len;
+  p->num_q_heads = num_q_heads;
+  p->workspace = static_cast<uint8_t*>(workspace);
+  p->workspace_bytes = workspace_bytes;
+  p->split_override = 0;
+  p->counters_off = kAlign;
+  p->counters_slots = counters_slots;
+  p->partial_off = kAlign + counters_bytes;
+  *out = p;
+  return ATLAS_OK;
+}
+
+atlas_status_t atlas_kv_pool_destroy(atlas_kv_pool_t* pool) {
+  delete pool;
+  return ATLAS_OK;
+}
+
+atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, int32_t split_tokens) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (split_tokens != 0 &&
+      (split_tokens < kMinSplit || split_tokens > kMaxSplit || split_tokens % kMinSplit != 0))
+    return ATLAS_ERR_INVALID_ARG;
+  pool->split_override = split_tokens;
+  return ATLAS_OK;
+}
+
+atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_new,
+                                   const void* v_new, int32_t dtype, const int32_t* block_table,
+                                   int32_t max_blocks_per_seq, const int32_t* start_pos,
+                                   int32_t batch, int32_t n_new, void* stream) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (batch < 0 || n_new < 0 || max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
+  if (dtype != ATLAS_DTYPE_F32 && dtype != ATLAS_DTYPE_BF16) return ATLAS_ERR_INVALID_ARG;
+  if (batch == 0 || n_new == 0) return ATLAS_OK;
+  if (!k_new || !v_new || !block_table || !start_pos) return ATLAS_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return ATLAS_ERR_INVALID_ARG;
+  atlas::AppendParams p;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.dtype = dtype;
+  p.k_pages = pool->k_pages;
+  p.v_pages = pool->v_pages;
+  p.k_scale = pool->k_scale;
+  p.v_scale = pool->v_scale;
+  p.block_table = block_table;
+  p.start_pos = start_pos;
+  p.err = reinterpret_cast<int32_t*>(pool->workspace);
+  p.batch = batch;
+  p.n_new = n_new;
+  p.Hkv = pool->num_kv_heads;
+  p.D = pool->head_dim;
+  p.ps = pool->page_size;
+  p.num_pages = pool->num_pages;
+  p.max_blocks = max_blocks_per_seq;
+  cudaError_t e = atlas::launch_fp8_append(p, device_sm_count(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+static atlas_status_t check_decode_shape(const atlas_kv_pool_t* pool, int32_t batch,
+                                         int32_t num_q_heads, int32_t q_len,
+                                         int32_t max_seq_len) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (batch < 0 || batch > pool->max_batch) return ATLAS_ERR_INVALID_ARG;
+  if (num_q_heads < 1 || num_q_heads % pool->num_kv_heads != 0) return ATLAS_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > pool->max_q_len) return ATLAS_ERR_INVALID_ARG;
+  if (max_seq_len < q_len) return ATLAS_ERR_INVALID_ARG;
+  return ATLAS_OK;
+}
+
+atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t batch,
+                                           int32_t num_q_heads, int32_t q_len,
+                                           int32_t max_seq_len, int32_t* plan, int32_t n) {
+  atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
+  if (st != ATLAS_OK) return st;
+  if (!plan || n < 0) return ATLAS_ERR_INVALID_ARG;
+  int sms = kDefaultSms;
+  {
+    int dev = 0, cnt = 0;
+    if (cudaGetDeviceCount(&cnt) == cudaSuccess && cnt > 0 && cudaGetDevice(&dev) == cudaSuccess)
+      sms = device_sm_count();
+    else
+      cudaGetLastError();
+  }
+  const Plan pl = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms);
+  const int32_t f[ATLAS_PLAN_FIELDS] = {pl.split_tokens, pl.num_splits, pl.kernel,
+                                        pl.rows_per_cta, pl.row_blocks, pl.launches,
+                                        (int32_t)(pl.grid_ctas > 0x7FFFFFFF ? 0x7FFFFFFF : pl.grid_ctas)};
+  for (int i = 0; i < n && i < ATLAS_PLAN_FIELDS; ++i) plan[i] = f[i];
+  return ATLAS_OK;
+}
+
+atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
+                                      const void* k_pages, const void* v_pages,
+                                      const float* k_scale, const float* v_scale,
+                                      const int32_t* block_table, int32_t max_blocks_per_seq,
+                                      const int32_t* seq_lens, int32_t batch,
+                                      int32_t num_q_heads, int32_t q_len, int32_t max_seq_len,
+                                      float sm_scale, void* out, void* stream) {
+  atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
+  if (st != ATLAS_OK) return st;
+  if (max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
+  if ((long long)max_seq_len > (long long)max_blocks_per_seq * pool->page_size)
+    return ATLAS_ERR_INVALID_ARG;
+  if (!(sm_scale == sm_scale) || isinf(sm_scale)) return ATLAS_ERR_INVALID_ARG;
+  if (batch == 0) return ATLAS_OK;
+  if (!q || !k_pages || !v_pages || !k_scale || !v_scale || !block_table || !seq_lens || !out)
+    return ATLAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return ATLAS_ERR_INVALID_ARG;
+
+  const int sms = device_sm_count();
+  const Plan pl = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms);
+  const int rows_all = q_len * num_q_heads;
+  if ((size_t)batch * pool->num_kv_heads * pl.row_blocks > pool->counters_slots)
+    return ATLAS_ERR_WORKSPACE;
+  if (pl.num_splits > 1 &&
+      pool->partial_off + partial_bytes(batch, pl.num_splits, rows_all, pool->head_dim) >
+          pool->workspace_bytes)
+    return ATLAS_ERR_WORKSPACE;
+  if (pl.num_splits > 65535 * 16 || batch > 65535) return ATLAS_ERR_UNSUPPORTED;
+
+  atlas::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pages = static_cast<const uint8_t*>(k_pages);
+  p.v_pages = static_cast<const uint8_t*>(v_pages);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  uint8_t* ws = pool->workspace;
+  p.err = reinterpret_cast<int32_t*>(ws);
+  p.counters = reinterpret_cast<int32_t*>(ws + pool->counters_off);
+  const size_t lse_bytes =
+      align_up((size_t)batch * pl.num_splits * rows_all * sizeof(float), kAlign);
+  p.part_lse = reinterpret_cast<float*>(ws + pool->partial_off);
+  p.part_o = reinterpret_cast<float*>(ws + pool->partial_off + lse_bytes);
+  p.B = batch;
+  p.Hq = num_q_heads;
+  p.Hkv = pool->num_kv_heads;
+  p.G = num_q_heads / pool->num_kv_heads;
+  p.q_len = q_len;
+  p.D = pool->head_dim;
+  p.ps = pool->page_size;
+  p.num_pages = pool->num_pages;
+  p.max_blocks = max_blocks_per_seq;
+  p.split_tokens = pl.split_tokens;
+  p.num_splits = pl.num_splits;
+  p.row_blocks = pl.row_blocks;
+  const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)pool->head_dim);
+  p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
+  cudaError_t e = atlas::launch_decode_mma(p, pl.rows_per_cta, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream, int32_t* code) {
+  if (!pool || !code) return ATLAS_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t host = 0;
+  if (cudaMemcpyAsync(&host, pool->workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return ATLAS_ERR_CUDA;
+  if (host != 0 && (cudaMemsetAsync(pool->workspace, 0, sizeof(int32_t), s) != cudaSuccess ||
+                    cudaStreamSynchronize(s) != cudaSuccess))
+    return ATLAS_ERR_CUDA;
+  *code = host;
+  return host == 0 ? ATLAS_OK : ATLAS_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

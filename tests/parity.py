@@ -1,0 +1,79 @@
+"""Helpers shared by the GPU parity tests: the oracle side of each check
+(computed only from the seeded generator's inputs, never from GPU output)
+and the tolerance rule."""
+
+import numpy as np
+
+from oracle import attention, e4m3, paged
+
+# Tolerance of the decode / verify output against the float64 oracle:
+# max-abs <= 1e-2 and relative L2 <= 5e-3 over the compared rows.  The bf16
+# store alone contributes up to 2^-9 relative per element.
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+
+
+def oracle_pages(w, which):
+    """uint8 pages the oracle expects after every token of every sequence of
+    workload ``w`` is appended (slots never written stay None-filled: use
+    the returned mask)."""
+    P, Hkv, ps, D = w.num_pages, w.num_kv_heads, w.page_size, w.head_dim
+    pages = np.zeros((P, Hkv, ps, D), np.uint8)
+    written = np.zeros((P, Hkv, ps), bool)
+    scale = w.k_scale if which == "k" else w.v_scale
+    src = w.k if which == "k" else w.v
+    for b in range(w.batch):
+        L = int(w.seq_lens[b])
+        codes = e4m3.encode(src[w.cu_seqlens[b]:w.cu_seqlens[b + 1]], scale[None, :, None])
+        t = np.arange(L)
+        pg = w.block_table[b, t // ps]
+        pages[pg, :, t % ps, :] = codes
+        written[pg, :, t % ps] = True
+    return pages, written
+
+
+def oracle_decode(w, sequences=None, sm_scale=None):
+    kp, _ = oracle_pages_subset(w, "k", sequences)
+    vp, _ = oracle_pages_subset(w, "v", sequences)
+    return attention.paged_gqa_decode(w.q_f64(), kp, vp, w.k_scale, w.v_scale, w.block_table,
+                                      w.seq_lens, w.q_len, w.page_size, sm_scale=sm_scale,
+                                      sequences=sequences)
+
+
+def oracle_pages_subset(w, which, sequences):
+    """Like :func:`oracle_pages` but only for the listed sequences."""
+    if sequences is None:
+        return oracle_pages(w, which)
+    P, Hkv, ps, D = w.num_pages, w.num_kv_heads, w.page_size, w.head_dim
+    pages = np.zeros((P, Hkv, ps, D), np.uint8)
+    scale = w.k_scale if which == "k" else w.v_scale
+    src = w.k if which == "k" else w.v
+    for b in sequences:
+        L = int(w.seq_lens[b])
+        codes = e4m3.encode(src[w.cu_seqlens[b]:w.cu_seqlens[b + 1]], scale[None, :, None])
+        t = np.arange(L)
+        pages[w.block_table[b, t // ps], :, t % ps, :] = codes
+    return pages, None
+
+
+def errors(got, ref):
+    """(max-abs, rel-L2) of ``got`` against ``ref`` over the finite rows of ref."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    sel = np.isfinite(ref)
+    d = got[sel] - ref[sel]
+    max_abs = float(np.max(np.abs(d))) if d.size else 0.0
+    den = float(np.linalg.norm(ref[sel]))
+    rel = float(np.linalg.norm(d) / den) if den > 0 else float(np.linalg.norm(d))
+    return max_abs, rel
+
+
+def assert_close(got, ref, what=""):
+    max_abs, rel = errors(got, ref)
+    assert np.all(np.isfinite(np.asarray(got, np.float64)[np.isfinite(ref)])), f"{what}: non-finite output"
+    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {max_abs:.3g}, rel-L2 {rel:.3g}"
+    return max_abs, rel
+
+
+__all__ = ["oracle_pages", "oracle_decode", "errors", "assert_close", "MAX_ABS", "REL_L2",
+           "paged"]

@@ -1,0 +1,194 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before anything is enqueued (CPU only: every call
+below that carries fake pointers also carries at least one invalid argument,
+so no kernel is ever launched on them)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_fp8_kv_05_b200 import build
+
+build.build()  # in-tree, no-op when up to date
+
+from paged_fp8_kv_05_b200 import atlas_kv as ak  # noqa: E402
+
+HEADER = os.path.join(build.ROOT, "include", "atlas_kv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(atlas_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("atlas_kv_pool_create", "atlas_fp8_kv_append", "atlas_paged_gqa_decode"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ak.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert missing == []
+    assert set(declared_functions()) == set(ak.EXPORTED)
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {ak.LIB_PATH}").read()
+    atlas_syms = sorted(set(re.findall(r"\b(atlas_[A-Za-z0-9_]+)\b", out)))
+    assert atlas_syms == declared_functions()
+
+
+def test_status_strings_and_version():
+    assert ak.status_string(0) == "ok"
+    assert "workspace" in ak.status_string(-3)
+    assert ak.version().count(".") == 2
+
+
+def test_workspace_bytes():
+    n = ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 256)
+    # header + counters + lse + O for 16 splits
+    assert n >= 256 + 32 * 32 * 4 + 32 * 16 * 32 * (128 + 1) * 4
+    assert ak.atlas_kv_workspace_bytes(32, 1, 32, 96, 4096) == 0        # head_dim
+    assert ak.atlas_kv_workspace_bytes(32, 0, 32, 128, 4096) == 0       # q_len
+    assert (ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 64)
+            > ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 256))
+
+
+class _Fake:
+    """A host buffer used only as an address; never dereferenced here."""
+
+    def __init__(self, n=1 << 16):
+        self.buf = ctypes.create_string_buffer(n + 512)
+        addr = ctypes.addressof(self.buf)
+        self.ptr = ctypes.c_void_p((addr + 255) // 256 * 256)
+
+
+F = _Fake()
+
+
+def _create(**kw):
+    args = dict(num_pages=64, page_size=16, num_kv_heads=2, head_dim=64, k=F.ptr, v=F.ptr,
+                ks=F.ptr, vs=F.ptr, max_batch=4, max_q_len=5, num_q_heads=8, ws=F.ptr,
+                ws_bytes=1 << 16)
+    args.update(kw)
+    h = ctypes.c_void_p()
+    st = ak._lib.atlas_kv_pool_create(ctypes.byref(h), args["num_pages"], args["page_size"],
+                                      args["num_kv_heads"], args["head_dim"], args["k"],
+                                      args["v"], args["ks"], args["vs"], args["max_batch"],
+                                      args["max_q_len"], args["num_q_heads"], args["ws"],
+                                      args["ws_bytes"])
+    return st, h
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(page_size=8), ak.ATLAS_ERR_UNSUPPORTED),
+    (dict(page_size=24), ak.ATLAS_ERR_UNSUPPORTED),
+    (dict(head_dim=96), ak.ATLAS_ERR_UNSUPPORTED),
+    (dict(num_pages=0), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(num_q_heads=7), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(k=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(ws=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), ak.ATLAS_ERR_WORKSPACE),
+    (dict(k=ctypes.c_void_p(F.ptr.value + 8)), ak.ATLAS_ERR_INVALID_ARG),
+])
+def test_pool_create_rejects(kw, status):
+    st, h = _create(**kw)
+    assert st == status and not h.value
+
+
+def test_pool_create_ok_and_plan_is_host_only():
+    st, h = _create()
+    assert st == ak.ATLAS_OK and h.value
+    try:
+        buf = (ctypes.c_int32 * 7)()
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 100, buf, 7) == ak.ATLAS_OK
+        plan = dict(zip(ak.PLAN_FIELDS, buf))
+        assert plan["split_tokens"] % 64 == 0 and plan["num_splits"] >= 1
+        assert plan["rows_per_cta"] == 8 and plan["row_blocks"] == 1 and plan["launches"] == 1
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 5, 100, buf, 7) == ak.ATLAS_OK
+        assert buf[3] == 16 and buf[4] == 2           # 5 x 4 rows -> two blocks of 16
+        assert ak._lib.atlas_kv_pool_set_split_tokens(h, 128) == ak.ATLAS_OK
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 1000, buf, 7) == ak.ATLAS_OK
+        assert buf[0] == 128 and buf[1] == 8
+        for bad in (-64, 32, 100, 16384):
+            assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 5, 8, 1, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 6, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
+    finally:
+        assert ak._lib.atlas_kv_pool_destroy(h) == ak.ATLAS_OK
+
+
+def _decode(h, **kw):
+    a = dict(q=F.ptr, kp=F.ptr, vp=F.ptr, ks=F.ptr, vs=F.ptr, bt=F.ptr, max_blocks=8,
+             sl=F.ptr, batch=2, hq=8, q_len=1, max_seq=100, sm=0.0, out=F.ptr)
+    a.update(kw)
+    return ak._lib.atlas_paged_gqa_decode(h, a["q"], a["kp"], a["vp"], a["ks"], a["vs"], a["bt"],
+                                          a["max_blocks"], a["sl"], a["batch"], a["hq"],
+                                          a["q_len"], a["max_seq"], a["sm"], a["out"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(out=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(bt=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(sl=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(q_len=0), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(q_len=6), ak.ATLAS_ERR_INVALID_ARG),              # > max_q_len
+    (dict(hq=7), ak.ATLAS_ERR_INVALID_ARG),                 # not a multiple of Hkv
+    (dict(batch=-1), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(batch=5), ak.ATLAS_ERR_INVALID_ARG),              # > max_batch
+    (dict(max_seq=129), ak.ATLAS_ERR_INVALID_ARG),          # > max_blocks * page_size
+    (dict(max_blocks=0), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(q_len=3, max_seq=2), ak.ATLAS_ERR_INVALID_ARG),   # max_seq_len < q_len
+    (dict(sm=float("nan")), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(q=ctypes.c_void_p(F.ptr.value + 2)), ak.ATLAS_ERR_INVALID_ARG),
+])
+def test_decode_rejects_before_launch(kw, status):
+    st, h = _create()
+    try:
+        assert _decode(h, **kw) == status
+    finally:
+        ak._lib.atlas_kv_pool_destroy(h)
+
+
+def test_decode_and_append_empty_batch_are_noops():
+    st, h = _create()
+    try:
+        assert _decode(h, batch=0, q=None, out=None) == ak.ATLAS_OK
+        assert ak._lib.atlas_fp8_kv_append(h, None, None, 0, None, 4, None, 0, 3, None) == ak.ATLAS_OK
+        assert ak._lib.atlas_fp8_kv_append(h, None, None, 0, None, 4, None, 2, 0, None) == ak.ATLAS_OK
+    finally:
+        ak._lib.atlas_kv_pool_destroy(h)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(k=None), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(dtype=7), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(max_blocks=0), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(n_new=-1), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(k=ctypes.c_void_p(F.ptr.value + 4)), ak.ATLAS_ERR_INVALID_ARG),
+])
+def test_append_rejects_before_launch(args, status):
+    st, h = _create()
+    a = dict(k=F.ptr, v=F.ptr, dtype=0, bt=F.ptr, max_blocks=4, sp=F.ptr, batch=2, n_new=3)
+    a.update(args)
+    try:
+        assert ak._lib.atlas_fp8_kv_append(h, a["k"], a["v"], a["dtype"], a["bt"], a["max_blocks"],
+                                           a["sp"], a["batch"], a["n_new"], None) == status
+    finally:
+        ak._lib.atlas_kv_pool_destroy(h)
+
+
+def test_null_pool_is_rejected_everywhere():
+    buf = (ctypes.c_int32 * 7)()
+    code = ctypes.c_int32()
+    assert ak._lib.atlas_paged_gqa_decode_plan(None, 1, 8, 1, 10, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
+    assert ak._lib.atlas_get_device_error(None, None, ctypes.byref(code)) == ak.ATLAS_ERR_INVALID_ARG
+    assert ak._lib.atlas_kv_pool_set_split_tokens(None, 0) == ak.ATLAS_ERR_INVALID_ARG
+    assert ak._lib.atlas_kv_pool_destroy(None) == ak.ATLAS_OK
+    assert _decode(None) == ak.ATLAS_ERR_INVALID_ARG
