@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--split-tokens", type=int, default=0, help="override the split size")
+    ap.add_argument("--stages", type=int, default=0, help="override the K/V staging depth")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -318,6 +319,8 @@ def ours(args):
     dw = DeviceWorkload(w, device=device)
     if args.split_tokens:
         dw.pool.set_split_tokens(args.split_tokens)
+    if args.stages:
+        dw.pool.set_option(ak.OPT_STAGES, args.stages)
     plan = dw.plan()
     b_dec, b_app = algorithmic_bytes(w)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)

@@ -82,6 +82,7 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
 #define ATLAS_DEVERR_PAGE_ID   0x1   /* decode: block-table entry outside [0, num_pages) */
 #define ATLAS_DEVERR_SEQ_LEN   0x2   /* decode: seq_len < q_len, > max_seq_len or > table */
 #define ATLAS_DEVERR_APPEND    0x4   /* append: position or page id out of range          */
+#define ATLAS_DEVERR_TIMEOUT   0x8   /* decode: a bounded wait for staged K/V ran out      */
 
 /* Fields of atlas_paged_gqa_decode_plan's output array. */
 #define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split                           */
@@ -134,6 +135,17 @@ ATLAS_API atlas_status_t atlas_kv_pool_destroy(atlas_kv_pool_t* pool);
  * [64, 8192].  Meant for tuning and for split-invariance tests.
  */
 ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, int32_t split_tokens);
+
+/* Tuning options for atlas_kv_pool_set_option. */
+#define ATLAS_OPT_SPLIT_TOKENS   1   /* same as atlas_kv_pool_set_split_tokens           */
+#define ATLAS_OPT_STAGES         2   /* K/V staging depth per warp: 0 = auto, 3 or 4      */
+
+/*
+ * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of
+ * range return ATLAS_ERR_INVALID_ARG and change nothing.
+ */
+ATLAS_API atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option,
+                                                  int32_t value);
 
 /*
  * FP8 page append (quantise + scatter), the cache-fill step.

@@ -26,6 +26,9 @@ ATLAS_DTYPE_BF16 = 1
 DEVERR_PAGE_ID = 0x1
 DEVERR_SEQ_LEN = 0x2
 DEVERR_APPEND = 0x4
+DEVERR_TIMEOUT = 0x8
+OPT_SPLIT_TOKENS = 1
+OPT_STAGES = 2
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 
@@ -48,6 +51,7 @@ _SIGNATURES = [
       _c_i32, _c_i32, _c_i32, _c_ptr, _c_size]),
     ("atlas_kv_pool_destroy", ctypes.c_int, [_c_ptr]),
     ("atlas_kv_pool_set_split_tokens", ctypes.c_int, [_c_ptr, _c_i32]),
+    ("atlas_kv_pool_set_option", ctypes.c_int, [_c_ptr, _c_i32, _c_i32]),
     ("atlas_fp8_kv_append", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_ptr]),
     ("atlas_paged_gqa_decode", ctypes.c_int,
@@ -150,6 +154,10 @@ class KVPool:
     def set_split_tokens(self, tokens: int):
         _check(_lib.atlas_kv_pool_set_split_tokens(self.handle, tokens),
                "atlas_kv_pool_set_split_tokens")
+
+    def set_option(self, option: int, value: int):
+        _check(_lib.atlas_kv_pool_set_option(self.handle, option, value),
+               "atlas_kv_pool_set_option")
 
     def device_error(self, stream=None) -> int:
         code = _c_i32(0)

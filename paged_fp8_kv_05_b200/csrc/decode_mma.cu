@@ -21,19 +21,29 @@
 // and the CTA that finishes a (b, h, rb) last -- found with one atomic
 // counter, no waiting -- merges the splits and resets the counter.
 //
-// Per 16-token unit a warp issues, per thread, 4 + 4 coalesced 16-byte loads
-// straight from the page into registers (no shared-memory staging: every
-// byte is used by exactly one thread), converts E4M3 -> f16 exactly with
-// cvt.rn.f16x2.e4m3x2, and runs both contractions on the tensor cores with
-// mma.sync m16n8k16 (f16 in, f32 accumulate), tokens on the M side:
+// K/V staging.  Each warp owns a ring of S shared-memory stages; one stage
+// holds the K and the V tile of one 16-token unit (16 rows x D bytes each),
+// brought in by two 2-D TMA tile loads (cp.async.bulk.tensor, no multicast)
+// whose completion is counted on the stage's mbarrier.  The warp keeps S-1
+// units in flight while it computes one, without spending registers on
+// prefetch.  The tiles land with the 128-byte (D = 128) or 64-byte (D = 64)
+// swizzle, which makes every fragment read below bank-conflict-free.
+//
+// Per unit the warp converts E4M3 -> f16 exactly with cvt.rn.f16x2.e4m3x2 and
+// runs both contractions on the tensor cores with mma.sync m16n8k16 (f16 in,
+// f32 accumulate), tokens on the M side:
 //   S^T[16 tok x 8 rows]  = K_tile[16 x D] . Q^T[D x 8]
 //   O^T[D x 8 rows]      += V_tile^T[D x 16] . P^T[16 x 8]
 // The head dimension is permuted consistently between K and Q (any
 // permutation leaves q.k unchanged) so each thread's K fragment is two
-// contiguous 16-byte slices of a token row; for V the thread's 16-byte slice
-// of one token is interleaved with the next token's by byte_perm to form the
+// 16-byte chunks of a token row; for V the thread's 16-byte chunk of one
+// token is interleaved with the next token's by byte_perm to form the
 // token-pair registers the A operand needs.  P moves from the S^T
 // accumulator layout to the PV B-operand layout with one movmatrix.trans.
+//
+// Every mbarrier wait is bounded (200 ms of wall clock); if one runs out the
+// kernel flags ATLAS_DEVERR_TIMEOUT, drains its outstanding loads with the same
+// bound and finishes without computing further units.
 #include <float.h>
 #include <math.h>
 
@@ -45,66 +55,101 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
-
-template <int D>
-struct VSlice;  // one thread's V bytes of one token: D/8 bytes
-template <>
-struct VSlice<128> {
-  uint4 v;
-  __device__ __forceinline__ uint32_t word(int i) const {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-  }
-  __device__ __forceinline__ void load(const uint8_t* p) { v = ld_stream16(p); }
-  __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
-};
-template <>
-struct VSlice<64> {
-  uint2 v;
-  __device__ __forceinline__ uint32_t word(int i) const { return i == 0 ? v.x : v.y; }
-  __device__ __forceinline__ void load(const uint8_t* p) { v = ld_stream8(p); }
-  __device__ __forceinline__ void zero() { v = make_uint2(0, 0); }
-};
+constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
+__device__ __forceinline__ uint32_t word_of(const uint2& v, int i) { return i == 0 ? v.x : v.y; }
 
 template <int D>
-struct Unit {
-  static constexpr int NCH = D / 64;  // 16-byte K slices per token per thread
-  uint4 k[2][NCH];                    // tokens g8 and g8 + 8
-  VSlice<D> v[4];                     // tokens 2c, 2c+1, 2c+8, 2c+9
+struct Frag;  // one warp-lane's share of a 16-token unit, read from the staged tiles
+template <>
+struct Frag<128> {
+  uint4 k[2][2];  // [token g8 | g8+8][head-dim chunk j]: bytes 64j + 16c .. +16
+  uint4 v[4];     // tokens 2c, 2c+1, 2c+8, 2c+9: head dims 16*g8 .. +16
+  __device__ __forceinline__ uint32_t kword(int t, int ks) const { return word_of(k[t][ks >> 2], ks & 3); }
+  __device__ __forceinline__ uint32_t vword(int q, int w) const { return word_of(v[q], w); }
+  __device__ __forceinline__ void zero_v(int q) { v[q] = make_uint4(0, 0, 0, 0); }
+  // 128-byte swizzle: 16-byte chunk index XOR (row & 7)
+  __device__ __forceinline__ void load(const uint8_t* kt, const uint8_t* vt, int g8, int c) {
+    const int ja = g8 & 1;  // odd rows read their chunks in the other order: no bank conflict
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int row = g8 + 8 * t;
+      const uint8_t* rb = kt + row * 128;
+      const uint4 a = *reinterpret_cast<const uint4*>(rb + ((((4 * ja) + c) ^ (row & 7)) << 4));
+      const uint4 b = *reinterpret_cast<const uint4*>(rb + ((((4 * (1 - ja)) + c) ^ (row & 7)) << 4));
+      k[t][0] = ja ? b : a;
+      k[t][1] = ja ? a : b;
+    }
+    const int rows[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      v[q] = *reinterpret_cast<const uint4*>(vt + rows[q] * 128 + ((g8 ^ (rows[q] & 7)) << 4));
+  }
+};
+template <>
+struct Frag<64> {
+  uint4 k[2][1];  // [token g8 | g8+8]: bytes 16c .. +16
+  uint2 v[4];     // tokens 2c, 2c+1, 2c+8, 2c+9: head dims 8*g8 .. +8
+  __device__ __forceinline__ uint32_t kword(int t, int ks) const { return word_of(k[t][0], ks & 3); }
+  __device__ __forceinline__ uint32_t vword(int q, int w) const { return word_of(v[q], w); }
+  __device__ __forceinline__ void zero_v(int q) { v[q] = make_uint2(0, 0); }
+  // 64-byte swizzle: 16-byte chunk index XOR ((row >> 1) & 3)
+  __device__ __forceinline__ void load(const uint8_t* kt, const uint8_t* vt, int g8, int c) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int row = g8 + 8 * t;
+      k[t][0] = *reinterpret_cast<const uint4*>(kt + row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
+    }
+    const int rows[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      v[q] = *reinterpret_cast<const uint2*>(vt + rows[q] * 64 +
+                                             ((((g8 >> 1) ^ ((rows[q] >> 1) & 3))) << 4) +
+                                             8 * (g8 & 1));
+  }
 };
 
-struct SmemLayout {
-  int pid_off, m_off, l_off, o_off, total_floats;
+// Dynamic shared memory: [ring: warps x S stages x (K tile, V tile)] [mbarriers]
+// [page ids]; the warp-combine buffers reuse the ring after the main loop.
+struct SmemPlan {
+  size_t ring, bars, pids, total;
 };
-
-__host__ __device__ inline SmemLayout smem_layout(int D, int RB, int split_tokens) {
-  SmemLayout s;
-  const int pid_slots = split_tokens / 16 + 2;
-  s.pid_off = 0;
-  s.m_off = (pid_slots + 3) & ~3;
-  s.l_off = s.m_off + kWarps * RB;
-  s.o_off = s.l_off + kWarps * RB;
-  s.total_floats = s.o_off + kWarps * RB * D;
-  return s;
+__host__ __device__ inline SmemPlan smem_plan(int D, int S, int split_tokens) {
+  SmemPlan sp;
+  sp.ring = 0;
+  sp.bars = (size_t)kWarps * S * 2 * 16 * D;
+  sp.pids = sp.bars + (size_t)kWarps * S * 8;
+  sp.total = sp.pids + (size_t)(split_tokens / 16 + 2) * 4 + 1024;  // + alignment slack
+  return sp;
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_kernel(const DecodeParams p) {
+template <int D, int NT, int S>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
+    paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV) {
   constexpr int RB = 8 * NT;   // query rows per CTA
-  constexpr int NCH = D / 64;  // K 16-byte slices per token per thread
+  constexpr int NCH = D / 64;  // 16-byte K chunks per token per thread
   constexpr int KS = D / 16;   // k-steps of QK^T
   constexpr int MT = D / 16;   // m-tiles of O^T (head dims)
   constexpr int VB = D / 8;    // V bytes per token per thread
+  constexpr int TILE = 16 * D; // bytes of one K (or V) unit tile
+  constexpr int STAGE = 2 * TILE;
+  static_assert((size_t)kWarps * S * STAGE >= (size_t)(2 * kWarps * RB + kWarps * RB * D) * 4,
+                "combine buffers must fit in the ring");
 
-  extern __shared__ float smem[];
-  const SmemLayout lay = smem_layout(D, RB, p.split_tokens);
-  int* s_pid = reinterpret_cast<int*>(smem + lay.pid_off);
-  float* s_m = smem + lay.m_off;
-  float* s_l = smem + lay.l_off;
-  float* s_o = smem + lay.o_off;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const SmemPlan sp = smem_plan(D, S, p.split_tokens);
+  uint8_t* ring = smem + sp.ring;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars);
+  int* s_pid = reinterpret_cast<int*>(smem + sp.pids);
+  float* s_m = reinterpret_cast<float*>(ring);  // after the main loop only
+  float* s_l = s_m + kWarps * RB;
+  float* s_o = s_l + kWarps * RB;
   __shared__ int s_is_last;
 
   const int tid = threadIdx.x;
@@ -147,6 +192,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
       pid = -1;
     }
     s_pid[i] = pid;
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) mbar_init(&bars[warp * S + s], 1);
+    fence_mbar_init();
   }
 
   // ---- Q fragments (B operand of S^T = K Q^T), bf16 -> f16 (exact in range)
@@ -205,65 +255,65 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 
-  __syncthreads();
+  __syncthreads();  // page ids and barrier init visible
 
+  // this warp's units: u = warp + kWarps * i, i < n_my
   const int n_units = (t_end - t_begin + 15) / 16;
-  const size_t head_stride = (size_t)p.ps * D;
+  const int n_my = (warp < n_units) ? (n_units - warp + kWarps - 1) / kWarps : 0;
 
-  auto load_unit = [&](int u, Unit<D>& x) {
-    const int t0 = t_begin + 16 * u;
+  auto unit_t0 = [&](int i) { return t_begin + 16 * (warp + kWarps * i); };
+  auto issue = [&](int i) {  // lane 0 only: stage i % S <- unit i
+    const int t0 = unit_t0(i);
+    uint64_t* bar = &bars[warp * S + i % S];
     const int pid = s_pid[t0 / p.ps - pg_begin];
-    if (pid < 0) return;  // skipped at compute time
-    const size_t off = ((size_t)pid * p.Hkv + h) * head_stride + (size_t)(t0 % p.ps) * D;
-    const uint8_t* kb = p.k_pages + off;
-    const uint8_t* vb = p.v_pages + off;
-#pragma unroll
-    for (int j = 0; j < NCH; ++j) {
-      x.k[0][j] = ld_stream16(kb + g8 * D + j * 64 + 16 * c);
-      x.k[1][j] = ld_stream16(kb + (g8 + 8) * D + j * 64 + 16 * c);
+    if (pid < 0) {  // bad page id: complete the phase with no data
+      mbar_arrive(bar);
+      return;
     }
-    x.v[0].load(vb + (2 * c) * D + VB * g8);
-    x.v[1].load(vb + (2 * c + 1) * D + VB * g8);
-    x.v[2].load(vb + (2 * c + 8) * D + VB * g8);
-    x.v[3].load(vb + (2 * c + 9) * D + VB * g8);
+    const int row = (pid * p.Hkv + h) * p.ps + (t0 % p.ps);
+    uint8_t* dst = ring + (size_t)(warp * S + i % S) * STAGE;
+    mbar_arrive_expect_tx(bar, STAGE);
+    tma_load_2d(dst, &tmK, 0, row, bar);
+    tma_load_2d(dst + TILE, &tmV, 0, row, bar);
   };
 
-  auto compute_unit = [&](int u, Unit<D>& x) {
-    const int t0 = t_begin + 16 * u;
-    if (s_pid[t0 / p.ps - pg_begin] < 0) return;  // bad page id: tokens skipped
-
-    // S^T = K . Q^T  (A3 dequant-to-f16 + A4)
-    float sacc[NT][4];
+  auto compute_unit = [&](int t0, Frag<D>& x) {
+    // S^T = K . Q^T  (A3 dequant-to-f16 + A4), two accumulation chains
+    float sacc[2][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sacc[ch][nt][0] = sacc[ch][nt][1] = sacc[ch][nt][2] = sacc[ch][nt][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       uint32_t a0, a1, a2, a3;
-      e4m3x4_to_f16x2x2(word_of(x.k[0][ks / 4], ks % 4), a0, a2);
-      e4m3x4_to_f16x2x2(word_of(x.k[1][ks / 4], ks % 4), a1, a3);
+      e4m3x4_to_f16x2x2(x.kword(0, ks), a0, a2);
+      e4m3x4_to_f16x2x2(x.kword(1, ks), a1, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_16816(sacc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+      for (int nt = 0; nt < NT; ++nt)
+        mma_16816(sacc[ks & 1][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
     }
-
-    // scale into the log2 domain, causal / tail mask (A5)
+    float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] *= scale2;
+      for (int e = 0; e < 4; ++e) sc[nt][e] = (sacc[0][nt][e] + sacc[1][nt][e]) * scale2;
+
+    // causal / tail mask (A5)
     if (t0 + 15 > min_lim) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int tok = t0 + g8 + ((e & 2) ? 8 : 0);
-          if (tok > lim[nt][e & 1]) sacc[nt][e] = -INFINITY;
+          if (tok > lim[nt][e & 1]) sc[nt][e] = -INFINITY;
         }
     }
     if (t0 + 16 > L) {  // tail of the last page: no V garbage may reach P*V
-      if (t0 + 2 * c >= L) x.v[0].zero();
-      if (t0 + 2 * c + 1 >= L) x.v[1].zero();
-      if (t0 + 2 * c + 8 >= L) x.v[2].zero();
-      if (t0 + 2 * c + 9 >= L) x.v[3].zero();
+      if (t0 + 2 * c >= L) x.zero_v(0);
+      if (t0 + 2 * c + 1 >= L) x.zero_v(1);
+      if (t0 + 2 * c + 8 >= L) x.zero_v(2);
+      if (t0 + 2 * c + 9 >= L) x.zero_v(3);
     }
 
     // online softmax (A6): row max over the 16 tokens, rescale, P
@@ -275,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
       float pv[4];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float mx = fmaxf(sacc[nt][e], sacc[nt][e + 2]);
+        float mx = fmaxf(sc[nt][e], sc[nt][e + 2]);
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
@@ -284,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
         alpha[nt][e] = fast_exp2(m_run[nt][e] - m_use);
         changed |= (m_new != m_run[nt][e]);
         m_run[nt][e] = m_new;
-        pv[e] = fast_exp2(sacc[nt][e] - m_use);
-        pv[e + 2] = fast_exp2(sacc[nt][e + 2] - m_use);
+        pv[e] = fast_exp2(sc[nt][e] - m_use);
+        pv[e + 2] = fast_exp2(sc[nt][e + 2] - m_use);
         l_run[nt][e] = l_run[nt][e] * alpha[nt][e] + pv[e] + pv[e + 2];
       }
       pb[nt][0] = movmatrix_trans(pack_f16x2(pv[0], pv[1]));  // tokens 0..7
@@ -309,25 +359,47 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
       const int wi = mt >> 1;
       const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
       uint32_t a0, a1, a2, a3;
-      e4m3x4_to_f16x2x2(__byte_perm(x.v[0].word(wi), x.v[1].word(wi), sel), a0, a1);
-      e4m3x4_to_f16x2x2(__byte_perm(x.v[2].word(wi), x.v[3].word(wi), sel), a2, a3);
+      e4m3x4_to_f16x2x2(__byte_perm(x.vword(0, wi), x.vword(1, wi), sel), a0, a1);
+      e4m3x4_to_f16x2x2(__byte_perm(x.vword(2, wi), x.vword(3, wi), sel), a2, a3);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) mma_16816(acc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }
   };
 
-  // ---- main loop: register double buffer, one unit in flight ahead
-  {
-    Unit<D> cur, nxt;
-    int u = warp;
-    if (u < n_units) load_unit(u, cur);
+  // ---- main loop over this warp's units through the TMA ring
+  if (lane == 0) {
+    for (int i = 0; i < S && i < n_my; ++i) issue(i);
+  }
+  int consumed = 0;
+  bool aborted = false;
 #pragma unroll 1
-    for (; u < n_units; u += kWarps) {
-      if (u + kWarps < n_units) load_unit(u + kWarps, nxt);
-      compute_unit(u, cur);
-      cur = nxt;
+  for (int i = 0; i < n_my; ++i) {
+    const int st = i % S;
+    if (!mbar_wait_bounded(&bars[warp * S + st], (uint32_t)((i / S) & 1), kWaitLimitNs)) {
+      aborted = true;
+      break;
+    }
+    consumed = i + 1;
+    const int t0 = unit_t0(i);
+    if (s_pid[t0 / p.ps - pg_begin] >= 0) {
+      const uint8_t* kt = ring + (size_t)(warp * S + st) * STAGE;
+      Frag<D> x;
+      x.load(kt, kt + TILE, g8, c);
+      compute_unit(t0, x);
+    }
+    __syncwarp();
+    if (lane == 0 && i + S < n_my) {
+      fence_proxy_async_smem();
+      issue(i + S);
     }
   }
+  if (__any_sync(kFull, aborted)) {
+    if (lane == 0) atomicOr(p.err, ATLAS_DEVERR_TIMEOUT);
+    // drain the loads still in flight (issued: i < min(n_my, consumed + S)), bounded
+    for (int i = consumed; i < n_my && i < consumed + S; ++i)
+      mbar_wait_bounded(&bars[warp * S + i % S], (uint32_t)((i / S) & 1), kWaitLimitNs);
+  }
+  __syncthreads();  // every warp is done with the ring: reuse it for the combine
 
   // ---- per-warp state to shared memory
 #pragma unroll
@@ -429,29 +501,39 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) paged_decode_mma_ke
   if (tid == 0) *counter = 0;  // ready for the next call on this stream
 }
 
-template <int D, int NT>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t stream) {
-  const SmemLayout lay = smem_layout(D, 8 * NT, p.split_tokens);
-  const size_t smem = (size_t)lay.total_floats * sizeof(float);
-  auto kern = paged_decode_mma_kernel<D, NT>;
+template <int D, int NT, int S>
+cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                     cudaStream_t stream) {
+  const size_t smem = smem_plan(D, S, p.split_tokens).total;
+  auto kern = paged_decode_mma_kernel<D, NT, S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_splits * p.row_blocks, p.Hkv, p.B);
-  kern<<<grid, kThreads, smem, stream>>>(p);
+  kern<<<grid, kThreads, smem, stream>>>(p, tmK, tmV);
   return cudaGetLastError();
+}
+
+template <int D, int NT>
+cudaError_t launch_s(const DecodeParams& p, int stages, const CUtensorMap& tmK,
+                     const CUtensorMap& tmV, cudaStream_t stream) {
+  if (stages == 3) return launch_t<D, NT, 3>(p, tmK, tmV, stream);
+  if (stages == 4) return launch_t<D, NT, 4>(p, tmK, tmV, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-size_t decode_mma_smem_bytes(int D, int rows_per_cta, int split_tokens) {
-  return (size_t)smem_layout(D, rows_per_cta, split_tokens).total_floats * sizeof(float);
+size_t decode_mma_smem_bytes(int D, int stages, int split_tokens) {
+  return smem_plan(D, stages, split_tokens).total;
 }
 
-cudaError_t launch_decode_mma(const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
-  if (p.D == 128 && rows_per_cta == 8) return launch_t<128, 1>(p, stream);
-  if (p.D == 128 && rows_per_cta == 16) return launch_t<128, 2>(p, stream);
-  if (p.D == 64 && rows_per_cta == 8) return launch_t<64, 1>(p, stream);
-  if (p.D == 64 && rows_per_cta == 16) return launch_t<64, 2>(p, stream);
+cudaError_t launch_decode_mma(const DecodeParams& p, int rows_per_cta, int stages,
+                              const CUtensorMap& tmK, const CUtensorMap& tmV,
+                              cudaStream_t stream) {
+  if (p.D == 128 && rows_per_cta == 8) return launch_s<128, 1>(p, stages, tmK, tmV, stream);
+  if (p.D == 128 && rows_per_cta == 16) return launch_s<128, 2>(p, stages, tmK, tmV, stream);
+  if (p.D == 64 && rows_per_cta == 8) return launch_s<64, 1>(p, stages, tmK, tmV, stream);
+  if (p.D == 64 && rows_per_cta == 16) return launch_s<64, 2>(p, stages, tmK, tmV, stream);
   return cudaErrorInvalidValue;
 }
 

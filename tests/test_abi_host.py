@@ -95,6 +95,7 @@ def _create(**kw):
     (dict(ws=None), ak.ATLAS_ERR_INVALID_ARG),
     (dict(ws_bytes=16), ak.ATLAS_ERR_WORKSPACE),
     (dict(k=ctypes.c_void_p(F.ptr.value + 8)), ak.ATLAS_ERR_INVALID_ARG),
+    (dict(num_pages=1 << 20, num_kv_heads=128, page_size=16), ak.ATLAS_ERR_UNSUPPORTED),
 ])
 def test_pool_create_rejects(kw, status):
     st, h = _create(**kw)
@@ -117,6 +118,9 @@ def test_pool_create_ok_and_plan_is_host_only():
         assert buf[0] == 128 and buf[1] == 8
         for bad in (-64, 32, 100, 16384):
             assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
+        for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 4, 0), (ak.OPT_STAGES, 0, 0),
+                             (ak.OPT_STAGES, 5, -1), (ak.OPT_SPLIT_TOKENS, 256, 0), (99, 1, -1)):
+            assert ak._lib.atlas_kv_pool_set_option(h, opt, val) == st
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 5, 8, 1, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 6, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
     finally:
