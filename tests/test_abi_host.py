@@ -95,7 +95,7 @@ def _create(**kw):
     (dict(ws=None), ak.ATLAS_ERR_INVALID_ARG),
     (dict(ws_bytes=16), ak.ATLAS_ERR_WORKSPACE),
     (dict(k=ctypes.c_void_p(F.ptr.value + 8)), ak.ATLAS_ERR_INVALID_ARG),
-    (dict(num_pages=1 << 20, num_kv_heads=128, page_size=16), ak.ATLAS_ERR_UNSUPPORTED),
+    (dict(num_pages=1 << 20, num_kv_heads=128, num_q_heads=128), ak.ATLAS_ERR_UNSUPPORTED),
 ])
 def test_pool_create_rejects(kw, status):
     st, h = _create(**kw)
