@@ -45,18 +45,22 @@ def attend(q_rows, K, V, limits, sm_scale):
 
 
 def paged_gqa_decode(q, k_pages, v_pages, k_scale, v_scale, block_table,
-                     seq_lens, q_len, page_size, sm_scale=None, sequences=None):
+                     seq_lens, q_len, page_size, sm_scale=None, sequences=None,
+                     k_layout="tok", v_layout="tok"):
     """float64 ``[B, q_len, Hq, D]`` reference output.
 
     ``q``: float64 ``[B, q_len, Hq, D]``; ``k_pages``/``v_pages``: uint8
     ``[P, Hkv, ps, D]``; scales float32 ``[Hkv]``; ``block_table`` int
     ``[B, max_blocks]``; ``seq_lens`` int ``[B]``.  ``sequences`` restricts the
     work to a subset of b (other rows are left NaN), for sampled checks.
+    ``k_layout`` / ``v_layout`` name the in-page order of each page array
+    (:mod:`oracle.paged`): ``"tok"`` ``[P, Hkv, ps, D]`` or ``"dim"``
+    ``[P, Hkv, D, ps]``.
     """
     q = np.asarray(q, dtype=np.float64)
     B, ql, Hq, D = q.shape
     assert ql == q_len
-    Hkv = k_pages.shape[1]
+    Hkv = np.asarray(k_pages).shape[1]
     assert Hq % Hkv == 0, "Hq must be a multiple of Hkv"
     G = Hq // Hkv
     if sm_scale is None or sm_scale <= 0:
@@ -66,8 +70,8 @@ def paged_gqa_decode(q, k_pages, v_pages, k_scale, v_scale, block_table,
         L = int(seq_lens[b])
         if L < q_len:
             raise ValueError(f"sequence {b}: seq_len {L} < q_len {q_len}")
-        K = paged.gather_dequant(k_pages, k_scale, block_table, b, L, page_size)
-        V = paged.gather_dequant(v_pages, v_scale, block_table, b, L, page_size)
+        K = paged.gather_dequant(k_pages, k_scale, block_table, b, L, page_size, k_layout)
+        V = paged.gather_dequant(v_pages, v_scale, block_table, b, L, page_size, v_layout)
         limits = [L - q_len + i for i in range(q_len)]
         for h in range(Hkv):
             for g in range(G):

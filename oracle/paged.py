@@ -1,20 +1,29 @@
 """The paged FP8 KV cache, as plain array indexing.  Test infrastructure only.
 
-Layout (the pages give none; this is the reading the whole build uses):
-pages are ``uint8[P, Hkv, ps, D]`` -- physical page, KV head, slot in page,
-head dimension.  Token position ``p`` of sequence ``b`` lives in physical page
-``block_table[b, p // ps]`` at slot ``p % ps``.  The block table is the
-fixed-size-block pool of the Atlas deep-dive (ainews.cool, "Memory
-architecture" paragraph: KV blocks preallocated in fixed sizes); the FP8 codes
-are those of the GB10 page's "paged FP8 KV cache" (ainews.surl.tw).
+Layouts (the pages give none; these are the readings the whole build uses).
+Token position ``p`` of sequence ``b`` lives in physical page
+``block_table[b, p // ps]`` at slot ``p % ps``.  Inside a page, one of two
+orders:
 
-The only place the layout is spelled out is :func:`slot_of`; everything else
-goes through it, so another layout would change that one function.
+* ``"tok"`` (token-major): ``uint8[P, Hkv, ps, D]`` -- page, KV head, slot,
+  head dimension.  The K pages use it.
+* ``"dim"`` (head-dim-major): ``uint8[P, Hkv, D, ps]`` -- page, KV head, head
+  dimension, slot; each head's page is the transpose of its token-major
+  form.  The V pages use it, so that the values of consecutive tokens for one
+  head dimension are adjacent bytes.
+
+The block table is the fixed-size-block pool of the Atlas deep-dive
+(ainews.cool, "Memory architecture" paragraph: KV blocks preallocated in
+fixed sizes); the FP8 codes are those of the GB10 page's "paged FP8 KV cache"
+(ainews.surl.tw).  The two layouts are spelled out only in :func:`slot_of`,
+:func:`_store` and :func:`gather_codes`.
 """
 
 import numpy as np
 
 from . import e4m3
+
+LAYOUTS = ("tok", "dim")
 
 
 def slot_of(block_table, b: int, pos: int, page_size: int):
@@ -22,14 +31,24 @@ def slot_of(block_table, b: int, pos: int, page_size: int):
     return int(block_table[b, pos // page_size]), pos % page_size
 
 
-def append(pages, new, scale, block_table, start_pos, page_size):
+def _store(out, page, slot, codes, layout):
+    """Write one token's codes ``[Hkv, D]`` into ``page`` at ``slot``."""
+    if layout == "tok":
+        out[page, :, slot, :] = codes
+    elif layout == "dim":
+        out[page, :, :, slot] = codes
+    else:
+        raise ValueError(layout)
+
+
+def append(pages, new, scale, block_table, start_pos, page_size, layout="tok"):
     """Return a copy of ``pages`` with the new tokens quantised and written.
 
     ``new``: float32 ``[B, n_new, Hkv, D]`` (bf16 inputs are passed as their
     exact float32 values); ``scale``: float32 ``[Hkv]``; ``start_pos[b]`` is the
     position of the first new token of sequence b.  Element (b, t, h, d) is
-    encoded as ``E4M3(fp32(x) / fp32(scale[h]))`` and stored at
-    ``pages[page, h, slot, d]`` with ``(page, slot) = slot_of(b, start_pos[b] + t)``.
+    encoded as ``E4M3(fp32(x) / fp32(scale[h]))`` and stored for token position
+    ``start_pos[b] + t`` in the given page layout.
     """
     out = np.array(pages, dtype=np.uint8, copy=True)
     new = np.asarray(new, dtype=np.float32)
@@ -38,24 +57,31 @@ def append(pages, new, scale, block_table, start_pos, page_size):
     for b in range(B):
         for t in range(n_new):
             page, slot = slot_of(block_table, b, int(start_pos[b]) + t, page_size)
-            out[page, :, slot, :] = e4m3.encode(new[b, t], scale[:, None])
+            _store(out, page, slot, e4m3.encode(new[b, t], scale[:, None]), layout)
     return out
 
 
-def gather_codes(pages, block_table, b: int, length: int, page_size: int):
+def gather_codes(pages, block_table, b: int, length: int, page_size: int, layout="tok"):
     """Contiguous codes ``uint8[length, Hkv, D]`` of sequence ``b``'s first
     ``length`` tokens, re-assembled page by page."""
     pages = np.asarray(pages)
     n_pages = (length + page_size - 1) // page_size
     ids = np.asarray(block_table[b, :n_pages], dtype=np.int64)
-    blocks = pages[ids]                       # [n_pages, Hkv, ps, D]
-    seq = blocks.transpose(0, 2, 1, 3)        # [n_pages, ps, Hkv, D]
-    seq = seq.reshape(n_pages * page_size, pages.shape[1], pages.shape[3])
+    blocks = pages[ids]
+    if layout == "tok":                       # [n_pages, Hkv, ps, D]
+        seq = blocks.transpose(0, 2, 1, 3)
+    elif layout == "dim":                     # [n_pages, Hkv, D, ps]
+        seq = blocks.transpose(0, 3, 1, 2)
+    else:
+        raise ValueError(layout)
+    hkv = seq.shape[2]
+    seq = seq.reshape(n_pages * page_size, hkv, seq.shape[3])
     return seq[:length]
 
 
-def gather_dequant(pages, scale, block_table, b: int, length: int, page_size: int):
+def gather_dequant(pages, scale, block_table, b: int, length: int, page_size: int,
+                   layout="tok"):
     """Dequantised float64 ``[length, Hkv, D]``: ``decode(code) * scale[h]``."""
-    codes = gather_codes(pages, block_table, b, length, page_size)
+    codes = gather_codes(pages, block_table, b, length, page_size, layout)
     scale = np.asarray(scale, dtype=np.float32).astype(np.float64)
     return e4m3.decode(codes) * scale[None, :, None]

@@ -217,3 +217,13 @@ def test_seq_len_below_q_len_is_rejected():
     c["seq_lens"] = np.array([2], np.int32)
     with pytest.raises(ValueError):
         attention.paged_gqa_decode(**c)
+
+
+def test_v_layout_dim_matches_token_major():
+    rng = np.random.default_rng(17)
+    c = _rand_case(rng, 2, 8, 2, 16, 4, [9, 14], 3)
+    base = attention.paged_gqa_decode(**c)
+    c2 = dict(c, v_pages=np.ascontiguousarray(c["v_pages"].transpose(0, 1, 3, 2)))
+    assert np.array_equal(attention.paged_gqa_decode(v_layout="dim", **c2), base)
+    c3 = dict(c, k_pages=np.ascontiguousarray(c["k_pages"].transpose(0, 1, 3, 2)))
+    assert np.array_equal(attention.paged_gqa_decode(k_layout="dim", **c3), base)

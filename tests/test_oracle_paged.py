@@ -73,3 +73,41 @@ def test_append_in_two_calls_equals_one_call():
     # the round trip is within half an E4M3 step (relative 1/16) of the input
     err = np.abs(back[:, 0] - new[0, :, 0])
     assert np.all(err <= np.abs(new[0, :, 0]) / 16 + 2.0 ** -10 * scale[0])
+
+
+def test_dim_major_layout_is_the_per_page_transpose():
+    rng = np.random.default_rng(21)
+    P, Hkv, ps, D = 7, 2, 4, 6
+    tok = rng.integers(0, 256, (P, Hkv, ps, D), dtype=np.uint8)
+    dim = np.ascontiguousarray(tok.transpose(0, 1, 3, 2))        # [P, Hkv, D, ps]
+    table = np.array([[3, 0, 6], [5, 1, -1]], dtype=np.int32)
+    for b, L in [(0, 11), (1, 6), (0, 1)]:
+        a = paged.gather_codes(tok, table, b, L, ps, "tok")
+        g = paged.gather_codes(dim, table, b, L, ps, "dim")
+        assert np.array_equal(a, g)
+        for t in range(L):                                         # explicit indexing
+            for h in range(Hkv):
+                for d in range(D):
+                    assert g[t, h, d] == dim[table[b][t // ps], h, d, t % ps]
+
+
+def test_append_dim_major_writes_one_column_per_token():
+    rng = np.random.default_rng(22)
+    P, Hkv, ps, D = 5, 2, 4, 8
+    pages = rng.integers(0, 256, (P, Hkv, D, ps), dtype=np.uint8)
+    table = np.array([[2, 4, 0]], dtype=np.int32)
+    new = rng.standard_normal((1, 6, Hkv, D)).astype(np.float32)
+    scale = np.array([0.02, 0.05], np.float32)
+    out = paged.append(pages, new, scale, table, np.array([3]), ps, layout="dim")
+    touched = np.zeros(pages.shape, bool)
+    for t in range(6):
+        pos = 3 + t
+        page, slot = table[0][pos // ps], pos % ps
+        for h in range(Hkv):
+            assert np.array_equal(out[page, h, :, slot], e4m3.encode(new[0, t, h], scale[h]))
+            touched[page, h, :, slot] = True
+    assert np.array_equal(out[~touched], pages[~touched])
+    # same tokens through the token-major layout give the transposed pages
+    tok = paged.append(np.ascontiguousarray(pages.transpose(0, 1, 3, 2)), new, scale, table,
+                       np.array([3]), ps, layout="tok")
+    assert np.array_equal(tok.transpose(0, 1, 3, 2), out)
