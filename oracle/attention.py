@@ -54,8 +54,8 @@ def paged_gqa_decode(q, k_pages, v_pages, k_scale, v_scale, block_table,
     ``[B, max_blocks]``; ``seq_lens`` int ``[B]``.  ``sequences`` restricts the
     work to a subset of b (other rows are left NaN), for sampled checks.
     ``k_layout`` / ``v_layout`` name the in-page order of each page array
-    (:mod:`oracle.paged`): ``"tok"`` ``[P, Hkv, ps, D]`` or ``"dim"``
-    ``[P, Hkv, D, ps]``.
+    (:mod:`oracle.paged`): ``"tok"`` ``[P, Hkv, ps, D]``, ``"grp16"``
+    ``[P, Hkv, ps/16, D, 16]`` or ``"dim"`` ``[P, Hkv, D, ps]``.
     """
     q = np.asarray(q, dtype=np.float64)
     B, ql, Hq, D = q.shape

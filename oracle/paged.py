@@ -2,15 +2,18 @@
 
 Layouts (the pages give none; these are the readings the whole build uses).
 Token position ``p`` of sequence ``b`` lives in physical page
-``block_table[b, p // ps]`` at slot ``p % ps``.  Inside a page, one of two
+``block_table[b, p // ps]`` at slot ``p % ps``.  Inside a page, one of three
 orders:
 
 * ``"tok"`` (token-major): ``uint8[P, Hkv, ps, D]`` -- page, KV head, slot,
   head dimension.  The K pages use it.
-* ``"dim"`` (head-dim-major): ``uint8[P, Hkv, D, ps]`` -- page, KV head, head
-  dimension, slot; each head's page is the transpose of its token-major
-  form.  The V pages use it, so that the values of consecutive tokens for one
-  head dimension are adjacent bytes.
+* ``"grp16"`` (16-slot groups, head-dim-major inside a group):
+  ``uint8[P, Hkv, ps // 16, D, 16]`` -- page, KV head, group of 16 slots,
+  head dimension, slot within the group.  The V pages use it: the values of
+  16 consecutive tokens for one head dimension are adjacent bytes, and every
+  16-token piece of a page is one contiguous block.
+* ``"dim"`` (head-dim-major): ``uint8[P, Hkv, D, ps]``; the same as
+  ``"grp16"`` when ps = 16.
 
 The block table is the fixed-size-block pool of the Atlas deep-dive
 (ainews.cool, "Memory architecture" paragraph: KV blocks preallocated in
@@ -23,7 +26,8 @@ import numpy as np
 
 from . import e4m3
 
-LAYOUTS = ("tok", "dim")
+LAYOUTS = ("tok", "grp16", "dim")
+GROUP = 16
 
 
 def slot_of(block_table, b: int, pos: int, page_size: int):
@@ -35,6 +39,8 @@ def _store(out, page, slot, codes, layout):
     """Write one token's codes ``[Hkv, D]`` into ``page`` at ``slot``."""
     if layout == "tok":
         out[page, :, slot, :] = codes
+    elif layout == "grp16":
+        out[page, :, slot // GROUP, :, slot % GROUP] = codes
     elif layout == "dim":
         out[page, :, :, slot] = codes
     else:
@@ -70,6 +76,9 @@ def gather_codes(pages, block_table, b: int, length: int, page_size: int, layout
     blocks = pages[ids]
     if layout == "tok":                       # [n_pages, Hkv, ps, D]
         seq = blocks.transpose(0, 2, 1, 3)
+    elif layout == "grp16":                   # [n_pages, Hkv, ps/16, D, 16]
+        seq = blocks.transpose(0, 2, 4, 1, 3)  # [n_pages, ps/16, 16, Hkv, D]
+        seq = seq.reshape(seq.shape[0], seq.shape[1] * GROUP, seq.shape[3], seq.shape[4])
     elif layout == "dim":                     # [n_pages, Hkv, D, ps]
         seq = blocks.transpose(0, 3, 1, 2)
     else:

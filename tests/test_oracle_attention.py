@@ -227,3 +227,9 @@ def test_v_layout_dim_matches_token_major():
     assert np.array_equal(attention.paged_gqa_decode(v_layout="dim", **c2), base)
     c3 = dict(c, k_pages=np.ascontiguousarray(c["k_pages"].transpose(0, 1, 3, 2)))
     assert np.array_equal(attention.paged_gqa_decode(k_layout="dim", **c3), base)
+    # ps = 4 has no full 16-slot group: use a 16-slot page for grp16
+    c4 = _rand_case(rng, 2, 8, 2, 16, 16, [9, 30], 2)
+    base4 = attention.paged_gqa_decode(**c4)
+    v = c4["v_pages"]                                              # [P, Hkv, 16, D]
+    g = np.ascontiguousarray(v.reshape(v.shape[0], v.shape[1], 1, 16, v.shape[3]).transpose(0, 1, 2, 4, 3))
+    assert np.array_equal(attention.paged_gqa_decode(v_layout="grp16", **dict(c4, v_pages=g)), base4)

@@ -111,3 +111,22 @@ def test_append_dim_major_writes_one_column_per_token():
     tok = paged.append(np.ascontiguousarray(pages.transpose(0, 1, 3, 2)), new, scale, table,
                        np.array([3]), ps, layout="tok")
     assert np.array_equal(tok.transpose(0, 1, 3, 2), out)
+
+
+def test_grp16_layout_groups_sixteen_slots_head_dim_major():
+    rng = np.random.default_rng(23)
+    P, Hkv, ps, D = 5, 2, 48, 8
+    tok = rng.integers(0, 256, (P, Hkv, ps, D), dtype=np.uint8)
+    grp = np.empty((P, Hkv, ps // 16, D, 16), np.uint8)
+    for s in range(ps):                                            # explicit construction
+        grp[:, :, s // 16, :, s % 16] = tok[:, :, s, :]
+    table = np.array([[4, 1, 3], [0, 2, -1]], dtype=np.int32)
+    for b, L in [(0, 130), (1, 49), (0, 16), (1, 1)]:
+        assert np.array_equal(paged.gather_codes(tok, table, b, L, ps, "tok"),
+                              paged.gather_codes(grp, table, b, L, ps, "grp16"))
+    new = rng.standard_normal((1, 20, Hkv, D)).astype(np.float32)
+    sc = np.array([0.03, 0.01], np.float32)
+    a = paged.append(grp, new, sc, table, np.array([40]), ps, layout="grp16")
+    t = paged.append(tok, new, sc, table, np.array([40]), ps, layout="tok")
+    for s in range(ps):
+        assert np.array_equal(a[:, :, s // 16, :, s % 16], t[:, :, s, :])
