@@ -13,7 +13,10 @@
  * paragraph).  The pages fix no layout, page size, scale granularity,
  * rounding or mask convention; the readings used here are:
  *
- *   pages        uint8 E4M3 codes, layout [num_pages][num_kv_heads][page_size][head_dim]
+ *   pages        uint8 E4M3 codes; K pages token-major
+ *                [num_pages][num_kv_heads][page_size][head_dim]; V pages in
+ *                16-slot groups, head-dim-major inside a group:
+ *                [num_pages][num_kv_heads][page_size/16][head_dim][16]
  *   block table  int32 [batch][max_blocks_per_seq]; token p of sequence b is in
  *                page block_table[b][p / page_size], slot p % page_size
  *   scales       one float32 per KV head for K and one for V (static)
@@ -87,7 +90,7 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
 /* Fields of atlas_paged_gqa_decode_plan's output array. */
 #define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split                           */
 #define ATLAS_PLAN_NUM_SPLITS    1   /* splits for max_seq_len                        */
-#define ATLAS_PLAN_KERNEL        2   /* 1 = warp-level mma.sync kernel                */
+#define ATLAS_PLAN_KERNEL        2   /* 1 = FP8 mma.sync kernel (E4M3 tensor cores)    */
 #define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) handled per CTA    */
 #define ATLAS_PLAN_ROW_BLOCKS    4   /* CTAs per (split, KV head, sequence)           */
 #define ATLAS_PLAN_LAUNCHES      5   /* kernel launches per decode call               */
@@ -109,8 +112,10 @@ ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, 
 
 /*
  * Describe a page pool.  num_pages >= 1; page_size a multiple of 16 and
- * <= 1024; head_dim 64 or 128; num_kv_heads >= 1.  k_pages / v_pages: device
- * uint8 [num_pages][num_kv_heads][page_size][head_dim], 16-byte aligned.
+ * <= 1024; head_dim 64 or 128; num_kv_heads >= 1.  k_pages: device uint8
+ * [num_pages][num_kv_heads][page_size][head_dim] (token-major); v_pages:
+ * device uint8 [num_pages][num_kv_heads][page_size/16][head_dim][16] (16-slot
+ * groups, head-dim-major inside a group); both 16-byte aligned.
  * k_scale / v_scale: device float32 [num_kv_heads] (used by append; decode
  * takes its own scale pointers).  max_batch, max_q_len, num_q_heads bound the
  * decode calls (they size the counter region).  workspace: device memory of
@@ -138,7 +143,7 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
 
 /* Tuning options for atlas_kv_pool_set_option. */
 #define ATLAS_OPT_SPLIT_TOKENS   1   /* same as atlas_kv_pool_set_split_tokens           */
-#define ATLAS_OPT_STAGES         2   /* K/V staging depth per warp: 0 = auto, 3 or 4      */
+#define ATLAS_OPT_STAGES         2   /* K/V staging depth per stream: 0 = auto, 2 or 3   */
 
 /*
  * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of

@@ -108,17 +108,20 @@ class KVPool:
     """A page pool (K and V page arrays, per-head scales, decode workspace).
 
     ``atlas_kv_pool_create`` on caller-owned torch buffers; the buffers live
-    as long as this object.  ``k_pages`` / ``v_pages`` are uint8
-    ``[num_pages, num_kv_heads, page_size, head_dim]``.
+    as long as this object.  ``k_pages`` is uint8
+    ``[num_pages, num_kv_heads, page_size, head_dim]`` (token-major) and
+    ``v_pages`` uint8 ``[num_pages, num_kv_heads, page_size // 16, head_dim, 16]``
+    (16-slot groups, head-dim-major inside a group).
     """
 
     def __init__(self, num_pages, page_size, num_kv_heads, head_dim, k_scale, v_scale, *,
                  max_batch, max_q_len, num_q_heads, max_seq_len, device="cuda",
                  min_split_tokens=256, k_pages=None, v_pages=None, fill=None):
         dev = torch.device(device)
-        shape = (num_pages, num_kv_heads, page_size, head_dim)
-        self.k_pages = k_pages if k_pages is not None else torch.empty(shape, dtype=torch.uint8, device=dev)
-        self.v_pages = v_pages if v_pages is not None else torch.empty(shape, dtype=torch.uint8, device=dev)
+        kshape = (num_pages, num_kv_heads, page_size, head_dim)   # token-major
+        vshape = (num_pages, num_kv_heads, page_size // 16, head_dim, 16)   # 16-slot groups
+        self.k_pages = k_pages if k_pages is not None else torch.empty(kshape, dtype=torch.uint8, device=dev)
+        self.v_pages = v_pages if v_pages is not None else torch.empty(vshape, dtype=torch.uint8, device=dev)
         if fill is not None:
             self.k_pages.fill_(fill)
             self.v_pages.fill_(fill)

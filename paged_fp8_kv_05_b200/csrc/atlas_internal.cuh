@@ -21,8 +21,8 @@ struct AppendParams {
   const void* k_new;          // [B][n_new][Hkv][D] f32 or bf16
   const void* v_new;
   int dtype;                  // ATLAS_DTYPE_*
-  uint8_t* k_pages;           // [P][Hkv][ps][D]
-  uint8_t* v_pages;
+  uint8_t* k_pages;           // [P][Hkv][ps][D]  (token-major)
+  uint8_t* v_pages;           // [P][Hkv][ps/16][D][16]  (16-slot groups, head-dim-major)
   const float* k_scale;       // [Hkv]
   const float* v_scale;
   const int32_t* block_table; // [B][max_blocks]
@@ -33,8 +33,8 @@ struct AppendParams {
 
 struct DecodeParams {
   const __nv_bfloat16* q;     // [B][q_len][Hq][D]
-  const uint8_t* k_pages;     // [P][Hkv][ps][D]
-  const uint8_t* v_pages;
+  const uint8_t* k_pages;     // [P][Hkv][ps][D]  (token-major)
+  const uint8_t* v_pages;     // [P][Hkv][ps/16][D][16]  (16-slot groups, head-dim-major)
   const float* k_scale;       // [Hkv]
   const float* v_scale;
   const int32_t* block_table; // [B][max_blocks]
@@ -51,13 +51,11 @@ struct DecodeParams {
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
 
-// rows_per_cta is 8 or 16, stages 3 or 4; grid = (num_splits * row_blocks, Hkv, B).
-// tmK / tmV: 2-D TMA maps of the K / V page arrays viewed as
-// [num_pages * Hkv * page_size rows][head_dim bytes], box 16 rows, swizzled.
-cudaError_t launch_decode_mma(const DecodeParams& p, int rows_per_cta, int stages,
-                              const CUtensorMap& tmK, const CUtensorMap& tmV,
+// FP8 tensor-core decode kernel.  rows_per_warp is 8 or 16 and rbg (warps that
+// share one K/V stream) 1, 2 or 4; stages 2 or 3.  grid = (num_splits *
+// row_blocks, Hkv, B) with row_blocks = ceil(q_len * G / (rows_per_warp * rbg)).
+cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
                               cudaStream_t stream);
-size_t decode_mma_smem_bytes(int D, int stages, int split_tokens);
 
 // ------------------------------------------------------------ device helpers
 
@@ -93,7 +91,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 // Transpose an 8x8 matrix of 16-bit elements held one b32 pair per thread.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t r;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
   return r;
 }
 
@@ -149,14 +147,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One bounded probe of an mbarrier phase; the thread may sleep up to
+// ~0.5 ms inside the instruction while the phase is still pending.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
       : "memory");
   return ok != 0;
 }
@@ -176,6 +176,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
   return true;
+}
+
+// 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completion counted on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // 2-D TMA tile load global -> shared, completion counted on `bar` (no multicast).

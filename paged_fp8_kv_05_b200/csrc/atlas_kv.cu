@@ -6,8 +6,6 @@
 
 #include <new>
 
-#include <cudaTypedefs.h>
-
 #include "atlas_internal.cuh"
 
 struct atlas_kv_pool {
@@ -53,40 +51,6 @@ int device_sm_count() {
   return cached[dev];
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to libcuda).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2-D map of a page array seen as [num_pages * Hkv * page_size rows][head_dim bytes],
-// 16-row boxes, swizzled so that the kernel's fragment reads are conflict-free.
-bool encode_page_map(CUtensorMap* map, const void* pages, const atlas_kv_pool* pool) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t rows = (cuuint64_t)pool->num_pages * pool->num_kv_heads * pool->page_size;
-  const cuuint64_t dims[2] = {(cuuint64_t)pool->head_dim, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)pool->head_dim};
-  const cuuint32_t box[2] = {(cuuint32_t)pool->head_dim, 16};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle sw =
-      pool->head_dim == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pages), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 size_t partial_bytes(int batch, int num_splits, int rows_all, int head_dim) {
   const size_t lse = align_up((size_t)batch * num_splits * rows_all * sizeof(float), kAlign);
   const size_t o = align_up((size_t)batch * num_splits * rows_all * head_dim * sizeof(float), kAlign);
@@ -95,6 +59,7 @@ size_t partial_bytes(int batch, int num_splits, int rows_all, int head_dim) {
 
 struct Plan {
   int split_tokens, num_splits, kernel, rows_per_cta, row_blocks, launches, stages;
+  int rows_per_warp, rbg;
   long long grid_ctas;
 };
 
@@ -110,7 +75,10 @@ Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
   const int G = num_q_heads / pool->num_kv_heads;
   const int R = q_len * G;
   pl.kernel = 1;
-  pl.rows_per_cta = (R <= 8) ? 8 : 16;
+  // query rows (q_len x group) per warp, and warps sharing one K/V stream
+  pl.rows_per_warp = (R <= 8) ? 8 : 16;
+  pl.rbg = (R <= 16) ? 1 : (R <= 32 ? 2 : 4);
+  pl.rows_per_cta = pl.rows_per_warp * pl.rbg;
   pl.row_blocks = (R + pl.rows_per_cta - 1) / pl.rows_per_cta;
   int T;
   if (pool->split_override > 0) {
@@ -130,7 +98,7 @@ Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
   pl.num_splits = (max_seq_len + T - 1) / T;
   if (pl.num_splits < 1) pl.num_splits = 1;
   pl.launches = 1;
-  pl.stages = pool->stages_override > 0 ? pool->stages_override : 3;
+  pl.stages = pool->stages_override > 0 ? pool->stages_override : (pl.rbg == 1 ? 2 : 3);
   pl.grid_ctas = (long long)pl.num_splits * pl.row_blocks * pool->num_kv_heads * batch;
   return pl;
 }
@@ -179,7 +147,6 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   if (!k_pages || !v_pages || !k_scale || !v_scale || !workspace) return ATLAS_ERR_INVALID_ARG;
   if (!aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(workspace, kAlign))
     return ATLAS_ERR_INVALID_ARG;
-  if ((long long)num_pages * num_kv_heads * page_size >= (1LL << 31)) return ATLAS_ERR_UNSUPPORTED;
   const size_t counters_slots = (size_t)max_batch * num_q_heads * max_q_len;
   const size_t counters_bytes = align_up(counters_slots * sizeof(int32_t), kAlign);
   if (workspace_bytes < kAlign + counters_bytes) return ATLAS_ERR_WORKSPACE;
@@ -227,7 +194,7 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
     case ATLAS_OPT_SPLIT_TOKENS:
       return atlas_kv_pool_set_split_tokens(pool, value);
     case ATLAS_OPT_STAGES:
-      if (value != 0 && value != 3 && value != 4) return ATLAS_ERR_INVALID_ARG;
+      if (value != 0 && value != 2 && value != 3) return ATLAS_ERR_INVALID_ARG;
       pool->stages_override = value;
       return ATLAS_OK;
   }
@@ -359,10 +326,7 @@ atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q
   p.row_blocks = pl.row_blocks;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)pool->head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
-  CUtensorMap tmK, tmV;
-  if (!encode_page_map(&tmK, k_pages, pool) || !encode_page_map(&tmV, v_pages, pool))
-    return ATLAS_ERR_CUDA;
-  cudaError_t e = atlas::launch_decode_mma(p, pl.rows_per_cta, pl.stages, tmK, tmV,
+  cudaError_t e = atlas::launch_decode_fp8(p, pl.rows_per_warp, pl.rbg, pl.stages,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

@@ -9,9 +9,13 @@
 // (cvt.rn.satfinite), sign of zero kept.  The result must be bit-exact with
 // that definition.
 //
+// Page layouts: K pages are token-major [P][Hkv][ps][D]; V pages are kept in
+// groups of 16 slots, head-dim-major inside a group: [P][Hkv][ps/16][D][16]
+// (16 consecutive tokens of one head dimension adjacent).
 // Memory-bound: per element 4 (f32) or 2 (bf16) bytes read, 1 byte written.
 // One thread owns 16 consecutive elements of one (sequence, token, head) row:
-// 64 B (or 32 B) of coalesced input and one 16-byte store into the page.
+// 64 B (or 32 B) of coalesced input, then one 16-byte store into a K page or
+// 16 byte stores (one per head dimension, 16 bytes apart) into a V page.
 #include "atlas_internal.cuh"
 
 namespace atlas {
@@ -78,9 +82,16 @@ __global__ void __launch_bounds__(256) fp8_append_kernel(const AppendParams p) {
       const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
       packed[w] = (lo & 0xFFFFu) | (hi << 16);
     }
-    uint8_t* dst = (which ? p.v_pages : p.k_pages) +
-                   (((size_t)page * p.Hkv + h) * p.ps + (pos % p.ps)) * p.D + 16 * j;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (!which) {
+      uint8_t* dst = p.k_pages + (((size_t)page * p.Hkv + h) * p.ps + (pos % p.ps)) * p.D + 16 * j;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    } else {
+      const int slot = pos % p.ps;
+      uint8_t* dst = p.v_pages + (((size_t)page * p.Hkv + h) * (p.ps / 16) + slot / 16) * (16 * p.D) +
+                     (size_t)(16 * j) * 16 + (slot % 16);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) dst[16 * k] = (uint8_t)(packed[k >> 2] >> (8 * (k & 3)));
+    }
   }
 }
 

@@ -14,9 +14,10 @@ REL_L2 = 5e-3
 
 
 def oracle_pages(w, which):
-    """uint8 pages the oracle expects after every token of every sequence of
-    workload ``w`` is appended (slots never written stay None-filled: use
-    the returned mask)."""
+    """Token-major uint8 pages ``[P, Hkv, ps, D]`` the oracle expects after
+    every token of every sequence of workload ``w`` is appended, and the mask
+    of written (page, head, slot) triples.  (The GPU keeps V in 16-slot
+    groups; tests bring it to token-major with :func:`v_token_major`.)"""
     P, Hkv, ps, D = w.num_pages, w.num_kv_heads, w.page_size, w.head_dim
     pages = np.zeros((P, Hkv, ps, D), np.uint8)
     written = np.zeros((P, Hkv, ps), bool)
@@ -30,6 +31,13 @@ def oracle_pages(w, which):
         pages[pg, :, t % ps, :] = codes
         written[pg, :, t % ps] = True
     return pages, written
+
+
+def v_token_major(v):
+    """``[P, Hkv, ps/16, D, 16]`` (16-slot groups) -> ``[P, Hkv, ps, D]``."""
+    v = np.asarray(v)
+    P, H, G, D, _ = v.shape
+    return v.transpose(0, 1, 2, 4, 3).reshape(P, H, G * 16, D)
 
 
 def oracle_decode(w, sequences=None, sm_scale=None):

@@ -95,7 +95,6 @@ def _create(**kw):
     (dict(ws=None), ak.ATLAS_ERR_INVALID_ARG),
     (dict(ws_bytes=16), ak.ATLAS_ERR_WORKSPACE),
     (dict(k=ctypes.c_void_p(F.ptr.value + 8)), ak.ATLAS_ERR_INVALID_ARG),
-    (dict(num_pages=1 << 20, num_kv_heads=128, num_q_heads=128), ak.ATLAS_ERR_UNSUPPORTED),
 ])
 def test_pool_create_rejects(kw, status):
     st, h = _create(**kw)
@@ -112,14 +111,14 @@ def test_pool_create_ok_and_plan_is_host_only():
         assert plan["split_tokens"] % 64 == 0 and plan["num_splits"] >= 1
         assert plan["rows_per_cta"] == 8 and plan["row_blocks"] == 1 and plan["launches"] == 1
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 5, 100, buf, 7) == ak.ATLAS_OK
-        assert buf[3] == 16 and buf[4] == 2           # 5 x 4 rows -> two blocks of 16
+        assert buf[3] == 32 and buf[4] == 1           # 5 x 4 rows: two warps of 16 share K/V
         assert ak._lib.atlas_kv_pool_set_split_tokens(h, 128) == ak.ATLAS_OK
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 1000, buf, 7) == ak.ATLAS_OK
         assert buf[0] == 128 and buf[1] == 8
         for bad in (-64, 32, 100, 16384):
             assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
-        for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 4, 0), (ak.OPT_STAGES, 0, 0),
-                             (ak.OPT_STAGES, 5, -1), (ak.OPT_SPLIT_TOKENS, 256, 0), (99, 1, -1)):
+        for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 2, 0), (ak.OPT_STAGES, 0, 0),
+                             (ak.OPT_STAGES, 4, -1), (ak.OPT_SPLIT_TOKENS, 256, 0), (99, 1, -1)):
             assert ak._lib.atlas_kv_pool_set_option(h, opt, val) == st
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 5, 8, 1, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 6, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
