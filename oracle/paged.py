@@ -9,9 +9,12 @@ orders:
   head dimension.  The K pages use it.
 * ``"grp16"`` (16-slot groups, head-dim-major inside a group):
   ``uint8[P, Hkv, ps // 16, D, 16]`` -- page, KV head, group of 16 slots,
-  head dimension, slot within the group.  The V pages use it: the values of
-  16 consecutive tokens for one head dimension are adjacent bytes, and every
-  16-token piece of a page is one contiguous block.
+  head dimension, byte position of the slot inside the group.  The V pages
+  use it: the values of 16 consecutive tokens for one head dimension are
+  adjacent bytes, and every 16-token piece of a page is one contiguous block.
+  Inside a group the slots are interleaved: slot t sits at byte
+  ``GROUP_POS[t] = 4*((t % 8) // 2) + 2*(t // 8) + t % 2``, so that bytes
+  4c..4c+3 hold slots 2c, 2c+1, 2c+8, 2c+9.
 * ``"dim"`` (head-dim-major): ``uint8[P, Hkv, D, ps]``; the same as
   ``"grp16"`` when ps = 16.
 
@@ -28,6 +31,7 @@ from . import e4m3
 
 LAYOUTS = ("tok", "grp16", "dim")
 GROUP = 16
+GROUP_POS = np.array([4 * ((t % 8) // 2) + 2 * (t // 8) + t % 2 for t in range(GROUP)])
 
 
 def slot_of(block_table, b: int, pos: int, page_size: int):
@@ -40,7 +44,7 @@ def _store(out, page, slot, codes, layout):
     if layout == "tok":
         out[page, :, slot, :] = codes
     elif layout == "grp16":
-        out[page, :, slot // GROUP, :, slot % GROUP] = codes
+        out[page, :, slot // GROUP, :, GROUP_POS[slot % GROUP]] = codes
     elif layout == "dim":
         out[page, :, :, slot] = codes
     else:
@@ -77,6 +81,7 @@ def gather_codes(pages, block_table, b: int, length: int, page_size: int, layout
     if layout == "tok":                       # [n_pages, Hkv, ps, D]
         seq = blocks.transpose(0, 2, 1, 3)
     elif layout == "grp16":                   # [n_pages, Hkv, ps/16, D, 16]
+        blocks = blocks[..., GROUP_POS]        # byte positions -> slot order
         seq = blocks.transpose(0, 2, 4, 1, 3)  # [n_pages, ps/16, 16, Hkv, D]
         seq = seq.reshape(seq.shape[0], seq.shape[1] * GROUP, seq.shape[3], seq.shape[4])
     elif layout == "dim":                     # [n_pages, Hkv, D, ps]

@@ -34,8 +34,8 @@ def oracle_pages(w, which):
 
 
 def v_token_major(v):
-    """``[P, Hkv, ps/16, D, 16]`` (16-slot groups) -> ``[P, Hkv, ps, D]``."""
-    v = np.asarray(v)
+    """``[P, Hkv, ps/16, D, 16]`` (16-slot groups, interleaved) -> ``[P, Hkv, ps, D]``."""
+    v = np.asarray(v)[..., paged.GROUP_POS]
     P, H, G, D, _ = v.shape
     return v.transpose(0, 1, 2, 4, 3).reshape(P, H, G * 16, D)
 

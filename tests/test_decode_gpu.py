@@ -7,6 +7,7 @@ import pytest
 import torch
 
 from oracle import attention
+from oracle.paged import GROUP_POS
 from paged_fp8_kv_05_b200 import build, workloads
 
 from parity import assert_close, errors, oracle_decode, oracle_pages
@@ -145,7 +146,7 @@ def test_mtp_rows_ignore_later_drafts(ak):
             for t in range(L - q_len + i + 1, L):
                 page, slot = int(w.block_table[b, t // 16]), t % 16
                 kp[page, :, slot, :] = 0x3C                 # K pages: token-major
-                vp[page, :, slot // 16, :, slot % 16] = 0xC4  # V pages: 16-slot groups
+                vp[page, :, slot // 16, :, int(GROUP_POS[slot % 16])] = 0xC4  # V: 16-slot groups
         got = ak.atlas_paged_gqa_decode(dw.pool, dw.q, dw.block_table, dw.seq_lens,
                                         w.max_seq_len, out=torch.empty_like(dw.q),
                                         k_pages=kp, v_pages=vp)

@@ -231,5 +231,7 @@ def test_v_layout_dim_matches_token_major():
     c4 = _rand_case(rng, 2, 8, 2, 16, 16, [9, 30], 2)
     base4 = attention.paged_gqa_decode(**c4)
     v = c4["v_pages"]                                              # [P, Hkv, 16, D]
-    g = np.ascontiguousarray(v.reshape(v.shape[0], v.shape[1], 1, 16, v.shape[3]).transpose(0, 1, 2, 4, 3))
+    g = np.empty((v.shape[0], v.shape[1], 1, v.shape[3], 16), np.uint8)
+    for t in range(16):
+        g[:, :, 0, :, paged.GROUP_POS[t]] = v[:, :, t, :]
     assert np.array_equal(attention.paged_gqa_decode(v_layout="grp16", **dict(c4, v_pages=g)), base4)

@@ -117,9 +117,13 @@ def test_grp16_layout_groups_sixteen_slots_head_dim_major():
     rng = np.random.default_rng(23)
     P, Hkv, ps, D = 5, 2, 48, 8
     tok = rng.integers(0, 256, (P, Hkv, ps, D), dtype=np.uint8)
+    # slot t of a group sits at this byte: bytes 4c..4c+3 hold slots 2c, 2c+1, 2c+8, 2c+9
+    where = {0: 0, 1: 1, 8: 2, 9: 3, 2: 4, 3: 5, 10: 6, 11: 7, 4: 8, 5: 9, 12: 10, 13: 11,
+             6: 12, 7: 13, 14: 14, 15: 15}
+    assert [where[t] for t in range(16)] == list(paged.GROUP_POS)
     grp = np.empty((P, Hkv, ps // 16, D, 16), np.uint8)
     for s in range(ps):                                            # explicit construction
-        grp[:, :, s // 16, :, s % 16] = tok[:, :, s, :]
+        grp[:, :, s // 16, :, where[s % 16]] = tok[:, :, s, :]
     table = np.array([[4, 1, 3], [0, 2, -1]], dtype=np.int32)
     for b, L in [(0, 130), (1, 49), (0, 16), (1, 1)]:
         assert np.array_equal(paged.gather_codes(tok, table, b, L, ps, "tok"),
@@ -129,4 +133,4 @@ def test_grp16_layout_groups_sixteen_slots_head_dim_major():
     a = paged.append(grp, new, sc, table, np.array([40]), ps, layout="grp16")
     t = paged.append(tok, new, sc, table, np.array([40]), ps, layout="tok")
     for s in range(ps):
-        assert np.array_equal(a[:, :, s // 16, :, s % 16], t[:, :, s, :])
+        assert np.array_equal(a[:, :, s // 16, :, where[s % 16]], t[:, :, s, :])
