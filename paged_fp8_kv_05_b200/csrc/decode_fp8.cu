@@ -32,10 +32,11 @@
 // Q: k-step s = 2j + hs of 32 dims reads bytes 64j + 16c + 8hs + {0..7} of a
 // token row (c = lane % 4), so each lane's K operand is two 16-byte chunks of a
 // token row.  V pages are kept in 16-slot groups, head-dim-major inside a group
-// ([D][16] bytes), so a V^T fragment (4 tokens of one head dim) is 4 adjacent
-// bytes; one ldmatrix.x4 fetches the A operand of a 16-dim m-tile for 32
-// tokens.  P leaves the S^T accumulator through movmatrix.trans and two quad
-// shuffles per register.
+// ([D][16] bytes, slots interleaved so that bytes 4c..4c+3 hold slots 2c, 2c+1,
+// 2c+8, 2c+9), so a V^T fragment is 4 adjacent bytes and one ldmatrix.x4
+// fetches the A operand of a 16-dim m-tile for 32 tokens.  P leaves the S^T
+// accumulator through movmatrix.trans, which hands each lane exactly those
+// four tokens of its row -- no shuffles.
 //
 // Work split and staging.  CTA (split s, KV head h, sequence b, row group)
 // owns the KV tokens [s*T, min((s+1)*T, L_b)) and RBG blocks of 8*NT query rows.
@@ -125,10 +126,11 @@ __device__ __forceinline__ void split_e4m3x4(uint32_t w0, uint32_t w1, uint32_t&
   lo = l0 | (l1 << 16);
 }
 
-// Byte mask keeping the tokens of a 4-token group [4c, 4c+4) below `nvalid`.
+// Byte mask of a V^T fragment word (bytes 4c..4c+3 of a 16-slot group row,
+// holding slots 2c, 2c+1, 2c+8, 2c+9) keeping the slots below `nvalid`.
 __device__ __forceinline__ uint32_t token_mask4(int nvalid, int c) {
-  const int k = nvalid - 4 * c;
-  return k >= 4 ? 0xFFFFFFFFu : (k <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - k))));
+  return (2 * c < nvalid ? 0x000000FFu : 0u) | (2 * c + 1 < nvalid ? 0x0000FF00u : 0u) |
+         (2 * c + 8 < nvalid ? 0x00FF0000u : 0u) | (2 * c + 9 < nvalid ? 0xFF000000u : 0u);
 }
 
 // ----------------------------------------------------------- shared memory plan
@@ -424,56 +426,35 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         }
     }
 
-    // online softmax (A6) over the 32 tokens; p = 2^(s - m + 8)
-    uint32_t pbhi[NT][2], pblo[NT][2];
-    bool changed = false;
-    float alpha[NT][2];
+    // online softmax (A6) over the 32 tokens, p = 2^(s - m + 8) with m the running
+    // reference of the row.  The reference only moves (exact row max, rescale of
+    // O and l) when a score exceeds it by more than 0.5, so p <= 2^8.5 < 448
+    // and the common step needs no cross-lane max.
+    bool need = false;
+    float lmax[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float pa[4], pb[4];
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float mx = fmaxf(fmaxf(sa[nt][e], sa[nt][e + 2]), fmaxf(sb[nt][e], sb[nt][e + 2]));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-        const float sc = scale2[nt][e];
-        const float m_new = fmaxf(m_run[nt][e], mx * sc);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[nt][e] = fast_exp2(m_run[nt][e] - m_use);
-        changed |= (m_new != m_run[nt][e]);
-        m_run[nt][e] = m_new;
-        const float off = 8.f - m_use;
-        pa[e] = fast_exp2(fmaf(sa[nt][e], sc, off));
-        pa[e + 2] = fast_exp2(fmaf(sa[nt][e + 2], sc, off));
-        pb[e] = fast_exp2(fmaf(sb[nt][e], sc, off));
-        pb[e + 2] = fast_exp2(fmaf(sb[nt][e + 2], sc, off));
-        l_run[nt][e] = fmaf(l_run[nt][e], alpha[nt][e], (pa[e] + pa[e + 2]) + (pb[e] + pb[e + 2]));
+        lmax[nt][e] = fmaxf(fmaxf(sa[nt][e], sa[nt][e + 2]), fmaxf(sb[nt][e], sb[nt][e + 2])) *
+                      scale2[nt][e];
+        need |= lmax[nt][e] > m_run[nt][e] + 0.5f;
       }
-      // P^T B operand: row g8, tokens 4c..4c+3 of tile A (b0) and of tile B (b1)
-      const uint32_t xa = movmatrix_trans(pack_f16x2(pa[0], pa[1]));  // toks 2c, 2c+1
-      const uint32_t ya = movmatrix_trans(pack_f16x2(pa[2], pa[3]));  // toks 8+2c, 9+2c
-      const uint32_t xb = movmatrix_trans(pack_f16x2(pb[0], pb[1]));
-      const uint32_t yb = movmatrix_trans(pack_f16x2(pb[2], pb[3]));
-      const int src0 = 4 * g8 + ((2 * c) & 3), src1 = 4 * g8 + ((2 * c + 1) & 3);
-      const bool lowc = c < 2;
-      uint32_t w0, w1, v0, v1;
-      {
-        const uint32_t x0 = __shfl_sync(kFull, xa, src0), y0 = __shfl_sync(kFull, ya, src0);
-        const uint32_t x1 = __shfl_sync(kFull, xa, src1), y1 = __shfl_sync(kFull, ya, src1);
-        w0 = lowc ? x0 : y0;
-        w1 = lowc ? x1 : y1;
-      }
-      {
-        const uint32_t x0 = __shfl_sync(kFull, xb, src0), y0 = __shfl_sync(kFull, yb, src0);
-        const uint32_t x1 = __shfl_sync(kFull, xb, src1), y1 = __shfl_sync(kFull, yb, src1);
-        v0 = lowc ? x0 : y0;
-        v1 = lowc ? x1 : y1;
-      }
-      split_e4m3x4(w0, w1, pbhi[nt][0], pblo[nt][0]);
-      split_e4m3x4(v0, v1, pbhi[nt][1], pblo[nt][1]);
-    }
-    if (__any_sync(kFull, changed)) {
+    if (__any_sync(kFull, need)) {
+      float alpha[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = lmax[nt][e];
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+          const float m_new = fmaxf(m_run[nt][e], mx);
+          alpha[nt][e] = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run[nt][e] - m_new);
+          m_run[nt][e] = m_new;
+          l_run[nt][e] *= alpha[nt][e];
+        }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -483,6 +464,29 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
           acc[mt][nt][2] *= alpha[nt][0];
           acc[mt][nt][3] *= alpha[nt][1];
         }
+    }
+    // P^T B operand for row g8: movmatrix leaves tokens (2c, 2c+1) and (8+2c, 9+2c)
+    // of a 16-token tile in this lane -- exactly the slots of V^T bytes 4c..4c+3
+    uint32_t pbhi[NT][2], pblo[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pa[4], pb[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float sc = scale2[nt][e];
+        const float off = 8.f - ((m_run[nt][e] == -INFINITY) ? 0.f : m_run[nt][e]);
+        pa[e] = fast_exp2(fmaf(sa[nt][e], sc, off));
+        pa[e + 2] = fast_exp2(fmaf(sa[nt][e + 2], sc, off));
+        pb[e] = fast_exp2(fmaf(sb[nt][e], sc, off));
+        pb[e + 2] = fast_exp2(fmaf(sb[nt][e + 2], sc, off));
+        l_run[nt][e] += (pa[e] + pa[e + 2]) + (pb[e] + pb[e + 2]);
+      }
+      const uint32_t xa = movmatrix_trans(pack_f16x2(pa[0], pa[1]));  // toks 2c, 2c+1
+      const uint32_t ya = movmatrix_trans(pack_f16x2(pa[2], pa[3]));  // toks 8+2c, 9+2c
+      const uint32_t xb = movmatrix_trans(pack_f16x2(pb[0], pb[1]));
+      const uint32_t yb = movmatrix_trans(pack_f16x2(pb[2], pb[3]));
+      split_e4m3x4(xa, ya, pbhi[nt][0], pblo[nt][0]);
+      split_e4m3x4(xb, yb, pbhi[nt][1], pblo[nt][1]);
     }
 
     // O^T += V^T . P^T (A7): m-tile mt = head dims 16mt + {g8, g8 + 8}

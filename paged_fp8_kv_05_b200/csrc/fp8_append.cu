@@ -11,7 +11,9 @@
 //
 // Page layouts: K pages are token-major [P][Hkv][ps][D]; V pages are kept in
 // groups of 16 slots, head-dim-major inside a group: [P][Hkv][ps/16][D][16]
-// (16 consecutive tokens of one head dimension adjacent).
+// (16 consecutive tokens of one head dimension adjacent), slot t of a group at
+// byte 4*((t%8)/2) + 2*(t/8) + t%2 (bytes 4c..4c+3 hold slots 2c, 2c+1, 2c+8,
+// 2c+9, the token order of the decode kernel's P fragments).
 // Memory-bound: per element 4 (f32) or 2 (bf16) bytes read, 1 byte written.
 // One thread owns 16 consecutive elements of one (sequence, token, head) row:
 // 64 B (or 32 B) of coalesced input, then one 16-byte store into a K page or
@@ -86,9 +88,10 @@ __global__ void __launch_bounds__(256) fp8_append_kernel(const AppendParams p) {
       uint8_t* dst = p.k_pages + (((size_t)page * p.Hkv + h) * p.ps + (pos % p.ps)) * p.D + 16 * j;
       *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     } else {
-      const int slot = pos % p.ps;
+      const int slot = pos % p.ps, t = slot % 16;
+      const int byte = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
       uint8_t* dst = p.v_pages + (((size_t)page * p.Hkv + h) * (p.ps / 16) + slot / 16) * (16 * p.D) +
-                     (size_t)(16 * j) * 16 + (slot % 16);
+                     (size_t)(16 * j) * 16 + byte;
 #pragma unroll
       for (int k = 0; k < 16; ++k) dst[16 * k] = (uint8_t)(packed[k >> 2] >> (8 * (k & 3)));
     }
