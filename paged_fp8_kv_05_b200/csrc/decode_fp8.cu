@@ -427,9 +427,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     }
 
     // online softmax (A6) over the 32 tokens, p = 2^(s - m + 8) with m the running
-    // reference of the row.  The reference only moves (exact row max, rescale of
-    // O and l) when a score exceeds it by more than 0.5, so p <= 2^8.5 < 448
-    // and the common step needs no cross-lane max.
+    // reference of the row.  A row's reference only moves (to the exact row max,
+    // rescaling its O and l) when one of its scores exceeds it by more than 0.5,
+    // so p <= 2^8.5 < 448 and the common step needs no cross-lane max.
     bool need = false;
     float lmax[NT][2];
 #pragma unroll
@@ -450,8 +450,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
           mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-          const float m_new = fmaxf(m_run[nt][e], mx);
-          alpha[nt][e] = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run[nt][e] - m_new);
+          // decided per row (mx is uniform over the row's lanes), so a row's
+          // reference -- and its bits -- never depend on the other rows
+          const bool move = mx > m_run[nt][e] + 0.5f;
+          const float m_new = move ? mx : m_run[nt][e];
+          alpha[nt][e] = move ? fast_exp2(m_run[nt][e] - m_new) : 1.f;
           m_run[nt][e] = m_new;
           l_run[nt][e] *= alpha[nt][e];
         }
