@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   uint8_t* ring = smem;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + SM::BARS);
   uint64_t* empty_bar = full_bar + NSTREAM * S;
-  int* s_pid = reinterpret_cast<int*>(smem + SM::PIDS);
+  int* s_piece = reinterpret_cast<int*>(smem + SM::PIDS);
   __shared__ int s_is_last;
 
   const int tid = threadIdx.x;
@@ -204,16 +204,23 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   const int t_end = min(t_begin + p.split_tokens, L);
   const int n_split_b = (L + p.split_tokens - 1) / p.split_tokens;
 
-  // ---- page ids of this split (A2: block-table gather), checked once
-  const int pg_begin = t_begin / p.ps;
-  const int pg_last = (t_end - 1) / p.ps;
-  for (int i = tid; i <= pg_last - pg_begin; i += kThreads) {
-    int pid = __ldg(p.block_table + (size_t)b * p.max_blocks + pg_begin + i);
+  // ---- A2, block-table gather: index of every 16-token piece of this split,
+  // counted in 16*D-byte blocks of the page arrays (-1 for a bad page id).
+  // Piece k holds tokens [t_begin + 16k, +16): page (t / ps), slot group
+  // (t % ps) / 16; the divisions happen here once, not per unit.
+  const int n_pieces = (t_end - t_begin + 15) / 16;
+  const int groups_per_page = p.ps / 16;
+  for (int k = tid; k < n_pieces; k += kThreads) {
+    const int t = t_begin + 16 * k;
+    const int pg = t / p.ps;
+    int pid = __ldg(p.block_table + (size_t)b * p.max_blocks + pg);
+    int piece = -1;
     if (pid < 0 || pid >= p.num_pages) {
       atomicOr(p.err, ATLAS_DEVERR_PAGE_ID);
-      pid = -1;
+    } else {
+      piece = (pid * p.Hkv + h) * groups_per_page + (t - pg * p.ps) / 16;
     }
-    s_pid[i] = pid;
+    s_piece[k] = piece;
   }
   if (tid < NSTREAM * S) {
     mbar_init(&full_bar[tid], 1);
@@ -321,32 +328,31 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   const int n_my = (stream < n_units) ? (n_units - stream + NSTREAM - 1) / NSTREAM : 0;
   const bool producer = (rbw == 0) && (lane == 0);
   auto unit_t0 = [&](int i) { return t_begin + kUnit * (stream + NSTREAM * i); };
-  auto tile_pid = [&](int t0) { return t0 < t_end ? s_pid[t0 / p.ps - pg_begin] : -1; };
+  // pieces of unit i: 2(stream + NSTREAM i) and the next one (if inside the split)
+  auto piece_of = [&](int k) { return k < n_pieces ? s_piece[k] : -1; };
 
-  const size_t kv_head = (size_t)p.ps * D;  // bytes of one head's page (K or V)
+  constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
   auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
     const int st = i % S;
-    const int t0 = unit_t0(i);
+    const int k = 2 * (stream + NSTREAM * i);
     uint64_t* bar = &full_bar[stream * S + st];
     uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
-    const int pa = tile_pid(t0), pb = tile_pid(t0 + 16);
+    const int pa = piece_of(k), pb = piece_of(k + 1);
     const uint32_t bytes = (pa >= 0 ? 2 * TILE : 0) + (pb >= 0 ? 2 * TILE : 0);
     if (bytes == 0) {
       mbar_arrive(bar);
       return;
     }
     mbar_arrive_expect_tx(bar, bytes);
-    // a 16-token piece of a head's page is TILE contiguous bytes in both layouts:
-    // K rows (slot0 .. slot0 + 15) x D, V group slot0 / 16 ([D][16])
+    // a 16-token piece is TILE contiguous bytes in both layouts: K rows
+    // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
     if (pa >= 0) {
-      const size_t off = ((size_t)pa * p.Hkv + h) * kv_head + (size_t)(t0 % p.ps) * D;
-      bulk_load(dst, p.k_pages + off, TILE, bar);
-      bulk_load(dst + 2 * TILE, p.v_pages + off, TILE, bar);
+      bulk_load(dst, p.k_pages + (size_t)pa * kPiece, TILE, bar);
+      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pa * kPiece, TILE, bar);
     }
     if (pb >= 0) {
-      const size_t off = ((size_t)pb * p.Hkv + h) * kv_head + (size_t)((t0 + 16) % p.ps) * D;
-      bulk_load(dst + TILE, p.k_pages + off, TILE, bar);
-      bulk_load(dst + 3 * TILE, p.v_pages + off, TILE, bar);
+      bulk_load(dst + TILE, p.k_pages + (size_t)pb * kPiece, TILE, bar);
+      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pb * kPiece, TILE, bar);
     }
   };
 
@@ -407,9 +413,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       }
   };
 
-  auto compute_unit = [&](int t0, const uint8_t* stage) {
-    const int nvA = (tile_pid(t0) >= 0) ? min(16, t_end - t0) : 0;
-    const int nvB = (tile_pid(t0 + 16) >= 0) ? min(16, t_end - t0 - 16) : 0;
+  auto compute_unit = [&](int i, const uint8_t* stage) {
+    const int t0 = unit_t0(i);
+    const int k = 2 * (stream + NSTREAM * i);
+    const int nvA = (piece_of(k) >= 0) ? min(16, t_end - t0) : 0;
+    const int nvB = (piece_of(k + 1) >= 0) ? min(16, t_end - t0 - 16) : 0;
     float sa[NT][4], sb[NT][4];
     qk_unit(stage, sa, sb);
 
@@ -493,16 +501,21 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     }
 
     // O^T += V^T . P^T (A7): m-tile mt = head dims 16mt + {g8, g8 + 8}
-    const uint32_t mA = tail ? token_mask4(nvA, c) : 0xFFFFFFFFu;
-    const uint32_t mB = tail ? token_mask4(nvB, c) : 0xFFFFFFFFu;
     const int mat = lane >> 3, mrow = lane & 7;
     const uint32_t vbase = smem_u32(stage + 2 * TILE + ((mat >> 1) ? TILE : 0)) +
                            (uint32_t)((8 * (mat & 1) + mrow) * 16);
+    uint32_t mA = 0xFFFFFFFFu, mB = 0xFFFFFFFFu;
+    if (tail) {  // slots past the end of the sequence (or of a skipped page)
+      mA = token_mask4(nvA, c);
+      mB = token_mask4(nvB, c);
+    }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4(vbase + mt * 256, a0, a1, a2, a3);
-      a0 &= mA; a1 &= mA; a2 &= mB; a3 &= mB;
+      if (tail) {
+        a0 &= mA; a1 &= mA; a2 &= mB; a3 &= mB;
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         mma_e4m3(acc[mt][nt], a0, a1, a2, a3, pbhi[nt][0], pbhi[nt][1]);
@@ -526,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       break;
     }
     consumed = i + 1;
-    if (row0 < Rtot) compute_unit(unit_t0(i), ring + (size_t)(stream * S + st) * STAGE);
+    if (row0 < Rtot) compute_unit(i, ring + (size_t)(stream * S + st) * STAGE);
     __syncwarp();
     if constexpr (RBG > 1) {
       if (lane == 0) mbar_arrive(&empty_bar[stream * S + st]);
