@@ -228,6 +228,48 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   }
   if (tid == 0) fence_mbar_init();
 
+  __syncthreads();  // page ids and barrier init visible
+
+  // this stream's units: u = stream + NSTREAM * i, i < n_my
+  const int n_units = (t_end - t_begin + kUnit - 1) / kUnit;
+  const int n_my = (stream < n_units) ? (n_units - stream + NSTREAM - 1) / NSTREAM : 0;
+  const bool producer = (rbw == 0) && (lane == 0);
+  auto unit_t0 = [&](int i) { return t_begin + kUnit * (stream + NSTREAM * i); };
+  // pieces of unit i: 2(stream + NSTREAM i) and the next one (if inside the split)
+  auto piece_of = [&](int k) { return k < n_pieces ? s_piece[k] : -1; };
+
+  constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
+  auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
+    const int st = i % S;
+    const int k = 2 * (stream + NSTREAM * i);
+    uint64_t* bar = &full_bar[stream * S + st];
+    uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
+    const int pa = piece_of(k), pb = piece_of(k + 1);
+    const uint32_t bytes = (pa >= 0 ? 2 * TILE : 0) + (pb >= 0 ? 2 * TILE : 0);
+    if (bytes == 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    mbar_arrive_expect_tx(bar, bytes);
+    // a 16-token piece is TILE contiguous bytes in both layouts: K rows
+    // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
+    if (pa >= 0) {
+      bulk_load(dst, p.k_pages + (size_t)pa * kPiece, TILE, bar);
+      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pa * kPiece, TILE, bar);
+    }
+    if (pb >= 0) {
+      bulk_load(dst + TILE, p.k_pages + (size_t)pb * kPiece, TILE, bar);
+      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pb * kPiece, TILE, bar);
+    }
+  };
+
+
+  // the first S units of every stream go out before the query is prepared,
+  // so their loads overlap the Q fetch and split below
+  if (producer) {
+    for (int i = 0; i < S && i < n_my; ++i) issue(i);
+  }
+
   // ---- Q^T fragments as E4M3 hi + lo with a per-row power-of-two scale
   // B operand of k-step s = 2j + hs: b0 = dims 64j+16c+8hs+{0..3}, b1 = +{4..7}.
   uint32_t qhi[NT][KSTEP][2], qlo[NT][KSTEP][2];
@@ -320,41 +362,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-
-  __syncthreads();  // page ids and barrier init visible
-
-  // this stream's units: u = stream + NSTREAM * i, i < n_my
-  const int n_units = (t_end - t_begin + kUnit - 1) / kUnit;
-  const int n_my = (stream < n_units) ? (n_units - stream + NSTREAM - 1) / NSTREAM : 0;
-  const bool producer = (rbw == 0) && (lane == 0);
-  auto unit_t0 = [&](int i) { return t_begin + kUnit * (stream + NSTREAM * i); };
-  // pieces of unit i: 2(stream + NSTREAM i) and the next one (if inside the split)
-  auto piece_of = [&](int k) { return k < n_pieces ? s_piece[k] : -1; };
-
-  constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
-  auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
-    const int st = i % S;
-    const int k = 2 * (stream + NSTREAM * i);
-    uint64_t* bar = &full_bar[stream * S + st];
-    uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
-    const int pa = piece_of(k), pb = piece_of(k + 1);
-    const uint32_t bytes = (pa >= 0 ? 2 * TILE : 0) + (pb >= 0 ? 2 * TILE : 0);
-    if (bytes == 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    mbar_arrive_expect_tx(bar, bytes);
-    // a 16-token piece is TILE contiguous bytes in both layouts: K rows
-    // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
-    if (pa >= 0) {
-      bulk_load(dst, p.k_pages + (size_t)pa * kPiece, TILE, bar);
-      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pa * kPiece, TILE, bar);
-    }
-    if (pb >= 0) {
-      bulk_load(dst + TILE, p.k_pages + (size_t)pb * kPiece, TILE, bar);
-      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pb * kPiece, TILE, bar);
-    }
-  };
 
   // this lane's K operand words of one 16-token K tile: rows g8 and g8 + 8,
   // 16-byte chunks 4j + c (D = 128: odd rows fetch their chunks in the other
@@ -524,10 +531,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     }
   };
 
-  // ---- main loop over this stream's units through the TMA ring
-  if (producer) {
-    for (int i = 0; i < S && i < n_my; ++i) issue(i);
-  }
+  // ---- main loop over this stream's units through the staging ring
   int consumed = 0;
   bool aborted = false;
 #pragma unroll 1
