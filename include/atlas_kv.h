@@ -194,6 +194,34 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, con
                                       void* stream);
 
 /*
+ * The same decode / MTP-verify attention as atlas_paged_gqa_decode, for callers
+ * that cannot allocate device memory for a workspace (code running inside a
+ * host framework that owns every allocation and hands over only input and
+ * output buffers, or a path that must not touch the allocator).  The pages
+ * have no counterpart; this entry point exists for such callers only.
+ *
+ * No pool and no workspace: the geometry is passed directly, and the scratch
+ * (split-KV partials, completion counters, error word) lives in one static
+ * device array of 8 MiB per GPU, held from library load until process exit.
+ * Nothing here allocates.  Arguments and layouts are those of
+ * atlas_paged_gqa_decode plus num_kv_heads, head_dim, page_size and num_pages.
+ * Every call shares the array: each call clears the counters and error word
+ * on its stream before the launch, and calls that overlap on the GPU race.
+ * When the split-KV partials would not fit, longer splits are used (down to
+ * one per sequence); a call whose counters do not fit, or that would need
+ * splits longer than 65536 tokens, returns ATLAS_ERR_WORKSPACE.  The first
+ * call on a device looks up the array's address with that device current;
+ * make it before any stream capture.  Invalid sequences still get zero rows
+ * and bad page ids are skipped, but no error word is reported.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_decode_noalloc(
+    const void* q, const void* k_pages, const void* v_pages, const float* k_scale,
+    const float* v_scale, const int32_t* block_table, int32_t max_blocks_per_seq,
+    const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t page_size, int32_t num_pages, int32_t q_len, int32_t max_seq_len,
+    float sm_scale, void* out, void* stream);
+
+/*
  * The launch plan a decode call with these arguments would use (host only,
  * no CUDA call).  Writes min(n, ATLAS_PLAN_FIELDS) int32 fields to plan.
  */

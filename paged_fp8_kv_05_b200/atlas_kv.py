@@ -57,6 +57,9 @@ _SIGNATURES = [
     ("atlas_paged_gqa_decode", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32,
       _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
+    ("atlas_paged_gqa_decode_noalloc", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_i32,
+      _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_plan", ctypes.c_int,
      [_c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.POINTER(_c_i32), _c_i32]),
     ("atlas_get_device_error", ctypes.c_int, [_c_ptr, _c_ptr, ctypes.POINTER(_c_i32)]),
@@ -201,6 +204,26 @@ def atlas_paged_gqa_decode(pool: KVPool, q, block_table, seq_lens, max_seq_len, 
                                        _ptr(seq_lens), B, Hq, q_len, int(max_seq_len),
                                        float(sm_scale), _ptr(out), _stream(stream)),
            "atlas_paged_gqa_decode")
+    return out
+
+
+def atlas_paged_gqa_decode_noalloc(q, k_pages, v_pages, k_scale, v_scale, block_table,
+                                   seq_lens, max_seq_len, out=None, sm_scale=0.0, stream=None):
+    """The no-allocation decode entry point (scratch in the library's static
+    device array).  Page arrays as in :class:`KVPool`; ``q``/``out`` bf16
+    ``[B, q_len, Hq, D]``."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and block_table.is_contiguous()
+    B, q_len, Hq, D = (int(x) for x in q.shape)
+    P, Hkv, ps, Dk = (int(x) for x in k_pages.shape)
+    assert Dk == D
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.atlas_paged_gqa_decode_noalloc(_ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                               _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+                                               int(block_table.shape[1]), _ptr(seq_lens), B, Hq,
+                                               Hkv, D, ps, P, q_len, int(max_seq_len),
+                                               float(sm_scale), _ptr(out), _stream(stream)),
+           "atlas_paged_gqa_decode_noalloc")
     return out
 
 
