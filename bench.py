@@ -3,7 +3,8 @@
 
 One step = the whole hot path over one batch: the FP8 append of the step's
 q_len new K/V tokens per sequence (quantise + scatter into the pages) and the
-paged decode / verify attention over every sequence's full context.  The
+paged decode / verify attention over every sequence's full context, run as
+one fused kernel (atlas_paged_gqa_append_decode).  The
 default workload is the LLaMA-3-8B-shaped decode layer (B=32, Hq=32, Hkv=8,
 D=128, page 16, context U[1024, 4096], q_len=1); ``--config`` selects another
 of the five named workloads.
@@ -11,8 +12,8 @@ of the five named workloads.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
 
 Timing: L2 is flushed (a 256 MiB write) before every step, outside the CUDA
-events that bracket the step; the decode kernel is also timed alone by an
-event pair on the stream it is launched on.  Under torchrun every rank runs an
+events that bracket the step (the step is one kernel, so the event pair on
+its stream times that kernel).  Under torchrun every rank runs an
 independent replica (the path has no exchange step), the timed region is
 bracketed by a barrier and a device synchronise, and the max over ranks is
 taken.  Rank 0 prints one JSON line.
@@ -334,30 +335,24 @@ def ours(args):
         raise SystemExit("device error flag set during warm-up")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clk:
         for k in range(K):
             flush.zero_()
-            e0, e1, e2 = evs[k]
+            e0, e1 = evs[k]
             e0.record(stream)
-            dw.append_new()
+            dw.step()            # one kernel: FP8 append of the new tokens + decode
             e1.record(stream)
-            dw.decode()
-            e2.record(stream)
         torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_ms = max_over_ranks(sum(step_ms), dist, device)
-    dec_total = max_over_ranks(sum(dec_ms), dist, device)
     ms_per_step = total_ms / K
-    dec_ms_avg = dec_total / K
-    launches = 2 * K    # one append + one decode launch per step (plan: 1 decode launch)
+    launches = K         # the fused step is one launch (plan: 1 launch per call)
     assert plan["launches"] == 1
 
     # end to end through the public API with pinned host buffers
@@ -365,14 +360,13 @@ def ours(args):
     k_h = torch.from_numpy(w.new_tokens("k")).pin_memory()
     v_h = torch.from_numpy(w.new_tokens("v")).pin_memory()
     sl_h = torch.from_numpy(w.seq_lens.astype(np.int32)).pin_memory()
-    st_h = torch.from_numpy((w.seq_lens - w.q_len).astype(np.int32)).pin_memory()
     bt_h = torch.from_numpy(np.ascontiguousarray(w.block_table)).pin_memory()
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, sl_h, st_h, bt_h))
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, sl_h, bt_h))
     d2h = out_h.numel() * out_h.element_size()
     q_d = torch.empty_like(dw.q)
     k_d, v_d = torch.empty_like(dw.k_new), torch.empty_like(dw.v_new)
-    sl_d, st_d = torch.empty_like(dw.seq_lens), torch.empty_like(dw.start_new)
+    sl_d = torch.empty_like(dw.seq_lens)
     bt_d = torch.empty_like(dw.block_table)
     out_d = torch.empty_like(dw.q)
     K_e2e = min(K, 200)
@@ -381,10 +375,10 @@ def ours(args):
         flush.zero_()
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for dst, src in ((q_d, q_h), (k_d, k_h), (v_d, v_h), (sl_d, sl_h), (st_d, st_h), (bt_d, bt_h)):
+        for dst, src in ((q_d, q_h), (k_d, k_h), (v_d, v_h), (sl_d, sl_h), (bt_d, bt_h)):
             dst.copy_(src, non_blocking=True)
-        ak.atlas_fp8_kv_append(dw.pool, k_d, v_d, bt_d, st_d)
-        ak.atlas_paged_gqa_decode(dw.pool, q_d, bt_d, sl_d, w.max_seq_len, out=out_d)
+        ak.atlas_paged_gqa_append_decode(dw.pool, k_d, v_d, q_d, bt_d, sl_d, w.max_seq_len,
+                                         out=out_d)
         out_h.copy_(out_d, non_blocking=True)
         z.record(stream)
         z.synchronize()
@@ -395,8 +389,8 @@ def ours(args):
         raise SystemExit("device error flag set during timing")
 
     peak, peak_kind = load_peaks()
-    achieved = b_dec / (dec_ms_avg * 1e-3) / 1e9
     step_bytes = b_dec + b_app
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
     tokens = world * w.batch * w.q_len / (ms_per_step * 1e-3)
     line = {
@@ -407,15 +401,14 @@ def ours(args):
         "data": "synthetic (seeded generator; random N(0,1) q/K/V, no weights)",
         "config": workload_config(w, args.config, b_dec, b_app, args),
         "tokens_per_s_per_layer": tokens,
-        "decode_us": dec_ms_avg * 1e3,
-        "append_us": max_over_ranks(sum(app_ms), dist, device) / K * 1e3,
+        "step_us": ms_per_step * 1e3,
         "plan": plan,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / 8000.0,
-                     "kernel": "paged_decode_mma_kernel (decode, launch-averaged)",
+                     "kernel": "paged_decode_fp8_kernel (fused append + decode, launch-averaged)",
                      "traffic": recorded_traffic(args.config),
-                     "algorithmic_bytes": b_dec,
+                     "algorithmic_bytes": step_bytes,
                      "algorithmic_flops": algorithmic_flops(w)},
         "e2e": {"value": world * step_bytes / (e2e_total / K_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "ms_per_step": e2e_total / K_e2e, "h2d_bytes_per_step": h2d,

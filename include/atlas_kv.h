@@ -194,6 +194,25 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, con
                                       void* stream);
 
 /*
+ * One decode / verify step in one kernel: the FP8 append of the q_len new
+ * tokens of every sequence (A0) fused with the attention (A1-A9).  Equivalent
+ * to atlas_fp8_kv_append(pool, k_new, v_new, dtype, block_table,
+ * max_blocks_per_seq, start_pos = seq_lens - q_len, batch, q_len) followed by
+ * atlas_paged_gqa_decode on the pool's pages and scales: the pages end up
+ * bit-identical and so does the output.  The CTA whose KV split holds a new
+ * token quantises and writes it, then reads it back with the rest of its split.
+ * k_new / v_new: device [batch][q_len][num_kv_heads][head_dim] of dtype, 16-byte
+ * aligned.  A new token whose page id is outside [0, num_pages) is not written
+ * and flags ATLAS_DEVERR_APPEND (and ATLAS_DEVERR_PAGE_ID for the decode).
+ * Other arguments and errors as atlas_paged_gqa_decode.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_append_decode(
+    const atlas_kv_pool_t* pool, const void* k_new, const void* v_new, int32_t dtype,
+    const void* q, const int32_t* block_table, int32_t max_blocks_per_seq,
+    const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t q_len,
+    int32_t max_seq_len, float sm_scale, void* out, void* stream);
+
+/*
  * The same decode / MTP-verify attention as atlas_paged_gqa_decode, for callers
  * that cannot allocate device memory for a workspace (code running inside a
  * host framework that owns every allocation and hands over only input and

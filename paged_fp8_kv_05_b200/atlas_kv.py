@@ -57,6 +57,9 @@ _SIGNATURES = [
     ("atlas_paged_gqa_decode", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32,
       _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
+    ("atlas_paged_gqa_append_decode", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_i32,
+      _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_noalloc", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_i32,
       _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
@@ -204,6 +207,27 @@ def atlas_paged_gqa_decode(pool: KVPool, q, block_table, seq_lens, max_seq_len, 
                                        _ptr(seq_lens), B, Hq, q_len, int(max_seq_len),
                                        float(sm_scale), _ptr(out), _stream(stream)),
            "atlas_paged_gqa_decode")
+    return out
+
+
+def atlas_paged_gqa_append_decode(pool: KVPool, k_new, v_new, q, block_table, seq_lens,
+                                  max_seq_len, out=None, sm_scale=0.0, stream=None):
+    """One fused step: append the q_len new tokens (``k_new``/``v_new``
+    ``[B, q_len, Hkv, D]`` f32 or bf16) at positions ``seq_lens - q_len`` and
+    decode.  Returns ``out`` (bf16 ``[B, q_len, Hq, D]``)."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and block_table.is_contiguous()
+    assert k_new.shape == v_new.shape and k_new.dtype == v_new.dtype
+    assert k_new.is_contiguous() and v_new.is_contiguous()
+    dtype = {torch.float32: ATLAS_DTYPE_F32, torch.bfloat16: ATLAS_DTYPE_BF16}[k_new.dtype]
+    B, q_len, Hq, D = (int(x) for x in q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.atlas_paged_gqa_append_decode(pool.handle, _ptr(k_new), _ptr(v_new), dtype,
+                                              _ptr(q), _ptr(block_table),
+                                              int(block_table.shape[1]), _ptr(seq_lens), B, Hq,
+                                              q_len, int(max_seq_len), float(sm_scale),
+                                              _ptr(out), _stream(stream)),
+           "atlas_paged_gqa_append_decode")
     return out
 
 

@@ -47,6 +47,11 @@ struct DecodeParams {
   int B, Hq, Hkv, G, q_len, D, ps, num_pages, max_blocks;
   int split_tokens, num_splits, row_blocks;
   float qk_scale_log2;        // sm_scale * log2(e); k_scale[h] is folded in per head
+  // fused append (A0): when k_new != nullptr the kernel first quantises and
+  // writes the q_len new tokens of each sequence, positions L - q_len .. L - 1
+  const void* k_new;          // [B][q_len][Hkv][D] f32 or bf16, or nullptr
+  const void* v_new;
+  int new_dtype;              // ATLAS_DTYPE_*
 };
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
@@ -118,6 +123,68 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p) {
   return r;
 }
 
+// ---- FP8 append helpers (shared by the append kernel and the fused decode)
+
+// 16 consecutive inputs (f32 or bf16) starting at element `elem`, as exact f32.
+__device__ __forceinline__ void load16_as_f32(const void* base, size_t elem, int dtype,
+                                              float (&x)[16]) {
+  if (dtype == ATLAS_DTYPE_F32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(p + i);
+      x[4 * i + 0] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 v = __ldg(p + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {  // bf16 -> f32 is exact: the bits move up 16
+        x[8 * i + 2 * k + 0] = __uint_as_float(w[k] << 16);
+        x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+  }
+}
+
+// E4M3(fp32(x) / fp32(scale)): IEEE round-to-nearest division (never a
+// reciprocal multiply), then round-to-nearest-even with saturation to +-448.
+// Returns the 16 codes packed little-endian in 4 words.
+__device__ __forceinline__ uint4 quantize16_e4m3(const float (&x)[16], float scale) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float y0 = __fdiv_rn(x[4 * i + 0], scale), y1 = __fdiv_rn(x[4 * i + 1], scale);
+    const float y2 = __fdiv_rn(x[4 * i + 2], scale), y3 = __fdiv_rn(x[4 * i + 3], scale);
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
+    w[i] = (lo & 0xFFFFu) | (hi << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Store 16 codes of head dims [16j, 16j + 16) of token slot `slot` of a head's
+// page.  K pages are token-major [P][Hkv][ps][D]; V pages are 16-slot groups,
+// head-dim-major inside a group, [P][Hkv][ps/16][D][16], with slot t of a group
+// at byte 4*((t%8)/2) + 2*(t/8) + t%2.
+__device__ __forceinline__ void store16_k(uint8_t* k_pages, size_t head_page, int D, int ps,
+                                          int slot, int j, uint4 codes) {
+  uint8_t* dst = k_pages + (head_page * ps + slot) * D + 16 * j;
+  *reinterpret_cast<uint4*>(dst) = codes;
+}
+__device__ __forceinline__ void store16_v(uint8_t* v_pages, size_t head_page, int D, int ps,
+                                          int slot, int j, uint4 codes) {
+  const int t = slot % 16;
+  const int byte = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
+  uint8_t* dst = v_pages + (head_page * (ps / 16) + slot / 16) * (16 * D) + (size_t)(16 * j) * 16 + byte;
+  const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+  for (int k = 0; k < 16; ++k) dst[16 * k] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
+}
+
 // ---- shared-memory addresses, mbarriers and TMA (single PTX instructions)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -135,6 +202,11 @@ __device__ __forceinline__ void fence_mbar_init() {
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders this thread's earlier global writes before later async-proxy reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

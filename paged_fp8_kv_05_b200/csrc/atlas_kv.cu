@@ -65,10 +65,11 @@ struct Plan {
 
 // Split-KV partition (A1).  The host sees only max_seq_len, so it sizes the
 // grid as if every sequence were that long; splits past a sequence's end exit
-// at once.  Target about two waves of 4 resident CTAs per SM, splits a multiple
-// of 64 tokens in [kMinSplit, kMaxSplit]; the chunk adapts to the sequence
-// length and the SM count, the "block size adapted to sequence length and
-// architecture" of the Atlas deep-dive's attention paragraph.
+// at once.  Target one wave of resident CTAs (3 per SM for the 8-row variant,
+// 2 for the 16-row ones), splits a multiple of 64 tokens in [256, kMaxSplit];
+// the chunk adapts to the sequence length and the SM count, the "block size
+// adapted to sequence length and architecture" of the Atlas deep-dive's
+// attention paragraph.
 Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len, int max_seq_len,
                int sms) {
   Plan pl;
@@ -85,7 +86,7 @@ Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
     T = pool->split_override;
   } else {
     const long long units = (long long)batch * pool->num_kv_heads * pl.row_blocks;
-    const long long target = (long long)sms * 4 * 2;
+    const long long target = (long long)sms * (pl.rows_per_warp == 8 ? 3 : 2);
     long long want = (target + units - 1) / (units > 0 ? units : 1);
     if (want < 1) want = 1;
     long long t = (max_seq_len + want - 1) / want;
@@ -211,7 +212,7 @@ atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_ne
   if (batch == 0 || n_new == 0) return ATLAS_OK;
   if (!k_new || !v_new || !block_table || !start_pos) return ATLAS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return ATLAS_ERR_INVALID_ARG;
-  atlas::AppendParams p;
+  atlas::AppendParams p{};
   p.k_new = k_new;
   p.v_new = v_new;
   p.dtype = dtype;
@@ -266,13 +267,16 @@ atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t 
   return ATLAS_OK;
 }
 
-atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
-                                      const void* k_pages, const void* v_pages,
-                                      const float* k_scale, const float* v_scale,
-                                      const int32_t* block_table, int32_t max_blocks_per_seq,
-                                      const int32_t* seq_lens, int32_t batch,
-                                      int32_t num_q_heads, int32_t q_len, int32_t max_seq_len,
-                                      float sm_scale, void* out, void* stream) {
+}  // extern "C"
+
+static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
+                                  const void* k_pages, const void* v_pages,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, int32_t max_blocks_per_seq,
+                                  const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                  int32_t q_len, int32_t max_seq_len, float sm_scale, void* out,
+                                  const void* k_new, const void* v_new, int32_t new_dtype,
+                                  void* stream) {
   atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
   if (st != ATLAS_OK) return st;
   if (max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
@@ -296,7 +300,7 @@ atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q
     return ATLAS_ERR_WORKSPACE;
   if (pl.num_splits > 65535 * 16 || batch > 65535) return ATLAS_ERR_UNSUPPORTED;
 
-  atlas::DecodeParams p;
+  atlas::DecodeParams p{};  // value-initialised: no fused append unless set
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_pages = static_cast<const uint8_t*>(k_pages);
   p.v_pages = static_cast<const uint8_t*>(v_pages);
@@ -326,9 +330,43 @@ atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q
   p.row_blocks = pl.row_blocks;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)pool->head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.new_dtype = new_dtype;
   cudaError_t e = atlas::launch_decode_fp8(p, pl.rows_per_warp, pl.rbg, pl.stages,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+
+extern "C" {
+
+atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
+                                      const void* k_pages, const void* v_pages,
+                                      const float* k_scale, const float* v_scale,
+                                      const int32_t* block_table, int32_t max_blocks_per_seq,
+                                      const int32_t* seq_lens, int32_t batch,
+                                      int32_t num_q_heads, int32_t q_len, int32_t max_seq_len,
+                                      float sm_scale, void* out, void* stream) {
+  return decode_impl(pool, q, k_pages, v_pages, k_scale, v_scale, block_table,
+                     max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len, max_seq_len,
+                     sm_scale, out, nullptr, nullptr, ATLAS_DTYPE_F32, stream);
+}
+
+atlas_status_t atlas_paged_gqa_append_decode(const atlas_kv_pool_t* pool, const void* k_new,
+                                             const void* v_new, int32_t dtype, const void* q,
+                                             const int32_t* block_table,
+                                             int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                             int32_t batch, int32_t num_q_heads, int32_t q_len,
+                                             int32_t max_seq_len, float sm_scale, void* out,
+                                             void* stream) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (dtype != ATLAS_DTYPE_F32 && dtype != ATLAS_DTYPE_BF16) return ATLAS_ERR_INVALID_ARG;
+  if (batch > 0 && (!k_new || !v_new)) return ATLAS_ERR_INVALID_ARG;
+  if (batch > 0 && (!aligned(k_new, 16) || !aligned(v_new, 16))) return ATLAS_ERR_INVALID_ARG;
+  return decode_impl(pool, q, pool->k_pages, pool->v_pages, pool->k_scale, pool->v_scale,
+                     block_table, max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len,
+                     max_seq_len, sm_scale, out, k_new, v_new, dtype, stream);
 }
 
 atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream, int32_t* code) {

@@ -204,6 +204,40 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   const int t_end = min(t_begin + p.split_tokens, L);
   const int n_split_b = (L + p.split_tokens - 1) / p.split_tokens;
 
+  // ---- A0, fused append: quantise and store the step's new tokens that fall in
+  // this split (positions L - q_len .. L - 1), then order those global writes
+  // before the bulk copies that read the pages back
+  if (p.k_new != nullptr) {
+    const int first_new = L - p.q_len;
+    const int a0 = max(t_begin, first_new);
+    const int n_tok = t_end - a0;
+    if (n_tok > 0) {
+      constexpr int CH = D / 16;
+      for (int idx = tid; idx < 2 * n_tok * CH; idx += kThreads) {
+        const int which = idx / (n_tok * CH);  // 0 = K, 1 = V
+        const int r = idx - which * n_tok * CH;
+        const int pos = a0 + r / CH, j = r % CH;
+        const int page = __ldg(p.block_table + (size_t)b * p.max_blocks + pos / p.ps);
+        if (page < 0 || page >= p.num_pages) {
+          atomicOr(p.err, ATLAS_DEVERR_APPEND);
+          continue;
+        }
+        float x[16];
+        load16_as_f32(which ? p.v_new : p.k_new,
+                      (((size_t)b * p.q_len + (pos - first_new)) * p.Hkv + h) * D + 16 * j,
+                      p.new_dtype, x);
+        const uint4 codes = quantize16_e4m3(x, __ldg((which ? p.v_scale : p.k_scale) + h));
+        const size_t head_page = (size_t)page * p.Hkv + h;
+        if (!which)
+          store16_k(const_cast<uint8_t*>(p.k_pages), head_page, D, p.ps, pos % p.ps, j, codes);
+        else
+          store16_v(const_cast<uint8_t*>(p.v_pages), head_page, D, p.ps, pos % p.ps, j, codes);
+      }
+      __threadfence();
+      fence_proxy_async_global();
+    }
+  }
+
   // ---- A2, block-table gather: index of every 16-token piece of this split,
   // counted in 16*D-byte blocks of the page arrays (-1 for a bad page id).
   // Piece k holds tokens [t_begin + 16k, +16): page (t / ps), slot group

@@ -134,7 +134,7 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, kAlign + counters_bytes, s) != cudaSuccess) return ATLAS_ERR_CUDA;
 
-  atlas::DecodeParams p;
+  atlas::DecodeParams p{};  // value-initialised: no fused append unless set
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_pages = static_cast<const uint8_t*>(k_pages);
   p.v_pages = static_cast<const uint8_t*>(v_pages);
@@ -162,6 +162,8 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   p.row_blocks = row_blocks;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
+  p.k_new = nullptr;  // decode only
+  p.v_new = nullptr;
   cudaError_t e = atlas::launch_decode_fp8(p, rows_per_warp, rbg, stages, s);
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

@@ -23,31 +23,6 @@
 namespace atlas {
 namespace {
 
-__device__ __forceinline__ void load16_as_f32(const void* base, size_t elem, int dtype,
-                                              float (&x)[16]) {
-  if (dtype == ATLAS_DTYPE_F32) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 v = __ldg(p + i);
-      x[4 * i + 0] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
-    }
-  } else {
-    const uint4* p = reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(base) + elem);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      uint4 v = __ldg(p + i);
-      uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {   // bf16 -> f32 is exact: the bits move up 16
-        x[8 * i + 2 * k + 0] = __uint_as_float(w[k] << 16);
-        x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-      }
-    }
-  }
-}
-
 __global__ void __launch_bounds__(256) fp8_append_kernel(const AppendParams p) {
   const int chunks = p.D / 16;
   const long long per_tensor = (long long)p.batch * p.n_new * p.Hkv * chunks;
@@ -71,30 +46,12 @@ __global__ void __launch_bounds__(256) fp8_append_kernel(const AppendParams p) {
     const size_t src_elem = ((((size_t)b * p.n_new + t) * p.Hkv + h) * p.D) + 16 * j;
     float x[16];
     load16_as_f32(which ? p.v_new : p.k_new, src_elem, p.dtype, x);
-    const float sc = __ldg((which ? p.v_scale : p.k_scale) + h);
-
-    uint32_t packed[4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float y0 = __fdiv_rn(x[4 * w + 0], sc);
-      const float y1 = __fdiv_rn(x[4 * w + 1], sc);
-      const float y2 = __fdiv_rn(x[4 * w + 2], sc);
-      const float y3 = __fdiv_rn(x[4 * w + 3], sc);
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(y2, y3), __NV_SATFINITE, __NV_E4M3);
-      packed[w] = (lo & 0xFFFFu) | (hi << 16);
-    }
-    if (!which) {
-      uint8_t* dst = p.k_pages + (((size_t)page * p.Hkv + h) * p.ps + (pos % p.ps)) * p.D + 16 * j;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    } else {
-      const int slot = pos % p.ps, t = slot % 16;
-      const int byte = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
-      uint8_t* dst = p.v_pages + (((size_t)page * p.Hkv + h) * (p.ps / 16) + slot / 16) * (16 * p.D) +
-                     (size_t)(16 * j) * 16 + byte;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) dst[16 * k] = (uint8_t)(packed[k >> 2] >> (8 * (k & 3)));
-    }
+    const uint4 codes = quantize16_e4m3(x, __ldg((which ? p.v_scale : p.k_scale) + h));
+    const size_t head_page = (size_t)page * p.Hkv + h;
+    if (!which)
+      store16_k(p.k_pages, head_page, p.D, p.ps, pos % p.ps, j, codes);
+    else
+      store16_v(p.v_pages, head_page, p.D, p.ps, pos % p.ps, j, codes);
   }
 }
 

@@ -63,9 +63,13 @@ class DeviceWorkload:
                                          max(self.w.max_seq_len, self.w.q_len),
                                          out=self.out if out is None else out, stream=stream)
 
-    def step(self, stream=None):
-        self.append_new(stream)
-        return self.decode(stream)
+    def step(self, stream=None, out=None):
+        """One fused step (A0-A9 in one kernel): append the q_len new tokens
+        and decode."""
+        return ak.atlas_paged_gqa_append_decode(
+            self.pool, self.k_new, self.v_new, self.q, self.block_table, self.seq_lens,
+            max(self.w.max_seq_len, self.w.q_len), out=self.out if out is None else out,
+            stream=stream)
 
     def plan(self):
         return ak.atlas_paged_gqa_decode_plan(self.pool, self.w.batch, self.w.num_q_heads,

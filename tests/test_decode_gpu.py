@@ -210,3 +210,36 @@ def test_empty_batch_is_a_noop(ak):
     out0 = torch.empty_like(q0)
     ak.atlas_paged_gqa_decode(dw.pool, q0, dw.block_table[:0], dw.seq_lens[:0], 10, out=out0)
     assert dw.pool.device_error() == 0
+
+
+FUSED_CASES = [
+    # (workload builder, split override): new tokens inside one piece, across a
+    # page and a split boundary, and the two named decode / verify shapes
+    (lambda: _case(3, 32, 8, 128, 16, [66, 200, 17], 5, seed=31), 64),
+    (lambda: _case(2, 16, 1, 128, 64, [130, 64], 3, seed=32), 64),
+    (lambda: workloads.config_workload(1), 0),
+    (lambda: workloads.config_workload(2), 0),
+]
+
+
+@pytest.mark.parametrize("case", range(len(FUSED_CASES)))
+def test_fused_step_equals_append_then_decode(ak, case):
+    make, split = FUSED_CASES[case]
+    w = make()
+    from paged_fp8_kv_05_b200.device_cache import DeviceWorkload
+    sep = DeviceWorkload(w, fill_cache=False)
+    fus = DeviceWorkload(w, fill_cache=False)
+    for dw in (sep, fus):
+        dw.fill_prefix()
+        if split:
+            dw.pool.set_split_tokens(split)
+    sep.append_new()
+    out_sep = sep.decode(out=torch.empty_like(sep.q))
+    out_fus = fus.step(out=torch.empty_like(fus.q))
+    torch.cuda.synchronize()
+    assert sep.pool.device_error() == 0 and fus.pool.device_error() == 0
+    assert torch.equal(sep.pool.k_pages, fus.pool.k_pages)
+    assert torch.equal(sep.pool.v_pages, fus.pool.v_pages)
+    assert torch.equal(out_sep.view(torch.int16), out_fus.view(torch.int16))
+    # and the fused step on its own matches the oracle
+    assert_close(out_fus.float().cpu().numpy(), oracle_decode(w), f"fused case {case}")
