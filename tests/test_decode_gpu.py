@@ -227,8 +227,8 @@ def test_fused_step_equals_append_then_decode(ak, case):
     make, split = FUSED_CASES[case]
     w = make()
     from paged_fp8_kv_05_b200.device_cache import DeviceWorkload
-    sep = DeviceWorkload(w, fill_cache=False)
-    fus = DeviceWorkload(w, fill_cache=False)
+    sep = DeviceWorkload(w, fill_cache=False, min_split_tokens=64)
+    fus = DeviceWorkload(w, fill_cache=False, min_split_tokens=64)
     for dw in (sep, fus):
         dw.fill_prefix()
         if split:
