@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--split-tokens", type=int, default=0, help="override the split size")
     ap.add_argument("--stages", type=int, default=0, help="override the K/V staging depth")
+    ap.add_argument("--waves", type=int, default=0, help="CTAs per resident CTA slot")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -322,6 +323,8 @@ def ours(args):
         dw.pool.set_split_tokens(args.split_tokens)
     if args.stages:
         dw.pool.set_option(ak.OPT_STAGES, args.stages)
+    if args.waves:
+        dw.pool.set_option(ak.OPT_WAVES, args.waves)
     plan = dw.plan()
     b_dec, b_app = algorithmic_bytes(w)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)

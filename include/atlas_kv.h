@@ -88,27 +88,30 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
 #define ATLAS_DEVERR_TIMEOUT   0x8   /* decode: a bounded wait for staged K/V ran out      */
 
 /* Fields of atlas_paged_gqa_decode_plan's output array. */
-#define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split                           */
-#define ATLAS_PLAN_NUM_SPLITS    1   /* splits for max_seq_len                        */
+#define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per CTA range (most any CTA gets)    */
+#define ATLAS_PLAN_NUM_SPLITS    1   /* most CTA ranges one max-length segment spans  */
 #define ATLAS_PLAN_KERNEL        2   /* 1 = FP8 mma.sync kernel (E4M3 tensor cores)    */
-#define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) handled per CTA    */
-#define ATLAS_PLAN_ROW_BLOCKS    4   /* CTAs per (split, KV head, sequence)           */
+#define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) per segment        */
+#define ATLAS_PLAN_ROW_BLOCKS    4   /* segments per (sequence, KV head)              */
 #define ATLAS_PLAN_LAUNCHES      5   /* kernel launches per decode call               */
-#define ATLAS_PLAN_GRID_CTAS     6   /* CTAs launched (empty splits exit at once)     */
+#define ATLAS_PLAN_GRID_CTAS     6   /* CTAs launched                                 */
 #define ATLAS_PLAN_FIELDS        7
 
 /*
  * Bytes of workspace a pool needs so that decode calls with batch <=
- * max_batch, q_len <= max_q_len, the given num_q_heads and head_dim and
- * max_seq_len <= max_seq_len fit, for any split size >= min_split_tokens
- * (<= 0 selects 64, the smallest split the library uses on its own).
+ * max_batch, q_len <= max_q_len, the given head counts and head_dim and
+ * max_seq_len <= max_seq_len fit with the automatic partition, and -- when
+ * min_split_tokens > 0 -- with any split override >= min_split_tokens.
  * The workspace holds the split-KV partial results (float32 O rows and
- * log-sum-exp values), one completion counter per (sequence, KV head, row
- * block) and the device error word.  Returns 0 for invalid arguments.
+ * log2-sum-exp values, one slot per segment plus one per CTA), one completion
+ * counter per segment (sequence, KV head, row block) and the device error
+ * word.  The figure depends on the SM count of the current device (148 if
+ * none is visible).  Returns 0 for invalid arguments.
  */
-ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t num_q_heads,
-                                int32_t head_dim, int32_t max_seq_len,
-                                int32_t min_split_tokens);
+ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t max_seq_len,
+                                          int32_t min_split_tokens);
 
 /*
  * Describe a page pool.  num_pages >= 1; page_size a multiple of 16 and
@@ -135,15 +138,22 @@ ATLAS_API atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** pool, int32_t nu
 ATLAS_API atlas_status_t atlas_kv_pool_destroy(atlas_kv_pool_t* pool);
 
 /*
- * Override the KV split size (tokens per split) of later decode calls; 0
- * restores the automatic choice.  Must be 0 or a multiple of 64 in
- * [64, 8192].  Meant for tuning and for split-invariance tests.
+ * Override the partition of later decode calls: CTA ranges of about
+ * split_tokens KV tokens (ceil(units / (split_tokens / 32)) CTAs, where units
+ * counts 32-token units as if every sequence were max_seq_len long); 0
+ * restores the automatic choice (one range per resident CTA).  Must be 0 or a
+ * multiple of 64 in [64, 8192].  Meant for tuning and for split-invariance
+ * tests.
  */
 ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, int32_t split_tokens);
 
 /* Tuning options for atlas_kv_pool_set_option. */
 #define ATLAS_OPT_SPLIT_TOKENS   1   /* same as atlas_kv_pool_set_split_tokens           */
 #define ATLAS_OPT_STAGES         2   /* K/V staging depth per stream: 0 = auto, 2 or 3   */
+#define ATLAS_OPT_WAVES          3   /* automatic grid: CTAs per resident CTA slot, 0 = 1, */
+                                     /* up to 8 (smaller ranges the hardware schedules    */
+                                     /* as slots free up); the workspace must hold the    */
+                                     /* extra partial slots (ATLAS_ERR_WORKSPACE if not)  */
 
 /*
  * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of
@@ -177,12 +187,17 @@ ATLAS_API atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const 
  * k_scale / v_scale: device float32 [num_kv_heads].  block_table: device
  * int32 [batch][max_blocks_per_seq]; only the first ceil(seq_len/page_size)
  * entries of a row are read.  seq_lens: device int32 [batch].
- * max_seq_len: host upper bound of seq_lens (sizes the split grid).
+ * max_seq_len: host upper bound of seq_lens (bounds the work of one CTA).
  * out: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
  * A sequence with seq_len < q_len, seq_len > max_blocks_per_seq*page_size or
  * seq_len > max_seq_len gets zero output rows and flags ATLAS_DEVERR_SEQ_LEN; a page id outside
  * [0, num_pages) is skipped (its tokens do not take part) and flags
  * ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
+ * Partition: the 32-token units of all (sequence, KV head, row block)
+ * segments are cut into equal contiguous ranges, one per CTA, so every CTA
+ * streams the same number of KV bytes whatever the length mix; a segment cut
+ * by a range boundary is merged by log-sum-exp by the CTA that finishes it
+ * last.  A wait that runs out (200 ms) flags ATLAS_DEVERR_TIMEOUT.
  */
 ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
                                       const void* k_pages, const void* v_pages,
@@ -199,8 +214,8 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, con
  * to atlas_fp8_kv_append(pool, k_new, v_new, dtype, block_table,
  * max_blocks_per_seq, start_pos = seq_lens - q_len, batch, q_len) followed by
  * atlas_paged_gqa_decode on the pool's pages and scales: the pages end up
- * bit-identical and so does the output.  The CTA whose KV split holds a new
- * token quantises and writes it, then reads it back with the rest of its split.
+ * bit-identical and so does the output.  Every CTA whose range holds a new
+ * token quantises and writes it, then reads it back with the rest of its range.
  * k_new / v_new: device [batch][q_len][num_kv_heads][head_dim] of dtype, 16-byte
  * aligned.  A new token whose page id is outside [0, num_pages) is not written
  * and flags ATLAS_DEVERR_APPEND (and ATLAS_DEVERR_PAGE_ID for the decode).
@@ -226,9 +241,9 @@ ATLAS_API atlas_status_t atlas_paged_gqa_append_decode(
  * atlas_paged_gqa_decode plus num_kv_heads, head_dim, page_size and num_pages.
  * Every call shares the array: each call clears the counters and error word
  * on its stream before the launch, and calls that overlap on the GPU race.
- * When the split-KV partials would not fit, longer splits are used (down to
- * one per sequence); a call whose counters do not fit, or that would need
- * splits longer than 65536 tokens, returns ATLAS_ERR_WORKSPACE.  The first
+ * When the split-KV partials of the balanced partition would not fit, the
+ * call runs one CTA per segment (no partials); a call that would then need a
+ * segment longer than 65536 tokens returns ATLAS_ERR_WORKSPACE.  The first
  * call on a device looks up the array's address with that device current;
  * make it before any stream capture.  Invalid sequences still get zero rows
  * and bad page ids are skipped, but no error word is reported.
@@ -241,8 +256,10 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode_noalloc(
     float sm_scale, void* out, void* stream);
 
 /*
- * The launch plan a decode call with these arguments would use (host only,
- * no CUDA call).  Writes min(n, ATLAS_PLAN_FIELDS) int32 fields to plan.
+ * The launch plan a decode call with these arguments would use.  With a CUDA
+ * device present it queries the kernel's occupancy (no launch, no memory
+ * traffic); without one it reports the plan for a 148-SM GPU.  Writes
+ * min(n, ATLAS_PLAN_FIELDS) int32 fields to plan.
  */
 ATLAS_API atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t batch,
                                            int32_t num_q_heads, int32_t q_len,
@@ -250,7 +267,9 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool
 
 /*
  * Wait for the stream, read the pool's device error word into *code and
- * clear it.  Returns ATLAS_OK if it was zero, ATLAS_ERR_DEVICE_CHECK if not.
+ * clear it (and, if it was set, the completion counters a call that stopped
+ * early may have left).  Returns ATLAS_OK if it was zero,
+ * ATLAS_ERR_DEVICE_CHECK if not.
  */
 ATLAS_API atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream,
                                       int32_t* code);

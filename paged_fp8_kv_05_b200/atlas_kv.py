@@ -29,6 +29,7 @@ DEVERR_APPEND = 0x4
 DEVERR_TIMEOUT = 0x8
 OPT_SPLIT_TOKENS = 1
 OPT_STAGES = 2
+OPT_WAVES = 3
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 
@@ -45,7 +46,7 @@ _c_size = ctypes.c_size_t
 _SIGNATURES = [
     ("atlas_version", ctypes.c_char_p, []),
     ("atlas_status_string", ctypes.c_char_p, [ctypes.c_int]),
-    ("atlas_kv_workspace_bytes", _c_size, [_c_i32] * 6),
+    ("atlas_kv_workspace_bytes", _c_size, [_c_i32] * 7),
     ("atlas_kv_pool_create", ctypes.c_int,
      [ctypes.POINTER(_c_ptr), _c_i32, _c_i32, _c_i32, _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
       _c_i32, _c_i32, _c_i32, _c_ptr, _c_size]),
@@ -104,10 +105,10 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, head_dim, max_seq_len,
-                             min_split_tokens=256) -> int:
-    return int(_lib.atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, head_dim,
-                                             max_seq_len, min_split_tokens))
+def atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, num_kv_heads, head_dim,
+                             max_seq_len, min_split_tokens=256) -> int:
+    return int(_lib.atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, num_kv_heads,
+                                             head_dim, max_seq_len, min_split_tokens))
 
 
 class KVPool:
@@ -133,8 +134,8 @@ class KVPool:
             self.v_pages.fill_(fill)
         self.k_scale = torch.as_tensor(k_scale, dtype=torch.float32).to(dev).contiguous()
         self.v_scale = torch.as_tensor(v_scale, dtype=torch.float32).to(dev).contiguous()
-        nbytes = atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, head_dim,
-                                          max_seq_len, min_split_tokens)
+        nbytes = atlas_kv_workspace_bytes(max_batch, max_q_len, num_q_heads, num_kv_heads,
+                                          head_dim, max_seq_len, min_split_tokens)
         if nbytes == 0:
             raise AtlasError(ATLAS_ERR_INVALID_ARG, "atlas_kv_workspace_bytes")
         self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)

@@ -40,12 +40,15 @@ struct DecodeParams {
   const int32_t* block_table; // [B][max_blocks]
   const int32_t* seq_lens;    // [B]
   __nv_bfloat16* out;         // [B][q_len][Hq][D]
-  float* part_o;              // [B][num_splits][q_len*Hq][D]   (split partials)
-  float* part_lse;            // [B][num_splits][q_len*Hq]       (log2-domain LSE)
+  float* part_o;              // [slots][rows_per_cta][D]  (partials of cut segments)
+  float* part_lse;            // [slots][rows_per_cta]     (log2-domain LSE)
   int32_t* counters;          // [B][Hkv][row_blocks], zero between calls
   int32_t* err;               // device error word
-  int B, Hq, Hkv, G, q_len, D, ps, num_pages, max_blocks;
-  int split_tokens, num_splits, row_blocks;
+  int B, Hq, Hkv, G, q_len, D, ps, num_pages, max_blocks, max_seq_len;
+  int row_blocks;
+  int max_units;              // most 32-token units one CTA is given
+  int max_portions;           // most segments one CTA's range meets
+  int per_segment;            // 1: CTA c = segment c (no partials); 0: balanced ranges
   float qk_scale_log2;        // sm_scale * log2(e); k_scale[h] is folded in per head
   // fused append (A0): when k_new != nullptr the kernel first quantises and
   // writes the q_len new tokens of each sequence, positions L - q_len .. L - 1
@@ -56,11 +59,92 @@ struct DecodeParams {
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
 
-// FP8 tensor-core decode kernel.  rows_per_warp is 8 or 16 and rbg (warps that
-// share one K/V stream) 1, 2 or 4; stages 2 or 3.  grid = (num_splits *
-// row_blocks, Hkv, B) with row_blocks = ceil(q_len * G / (rows_per_warp * rbg)).
+// Launch shape of the decode kernel for one call (A1).  A segment is
+// (sequence, KV head, row group of rows_per_cta query rows); a unit is 32 KV
+// tokens of a segment.  Balanced mode: the units of all segments, in (b, h, rg)
+// order, are cut into `grid` equal ranges, one per CTA; a segment cut by a
+// range boundary leaves one partial per CTA it meets, merged by the CTA that
+// finishes it last.  Per-segment mode: one CTA per segment, no partials.
+struct DecodeLaunch {
+  int rows_per_warp, rbg, rows_per_cta, row_blocks, stages;
+  int waves;             // automatic grid: this many CTAs per resident CTA slot
+  long long segs;        // B * Hkv * row_blocks
+  long long units_max;   // segs * ceil(max_seq_len / 32): units if every L were max_seq_len
+  long long grid;        // CTAs
+  int max_units;         // units of the largest range
+  int max_portions;      // segments the largest range can meet
+  int per_segment;
+  long long slots;       // partial slots: segs + grid (0 in per-segment mode)
+};
+
+constexpr int kMaxUnitsPerCta = 1024;  // bounds the per-CTA unit table in shared memory
+
+// Resident CTAs per SM the kernel is built for (its __launch_bounds__).
+inline int decode_target_occupancy(int rows_per_warp, int rbg) {
+  return (rows_per_warp <= 8 && rbg == 1) ? 3 : 2;
+}
+
+// split_tokens > 0: ranges of about split_tokens KV tokens (a multiple of 32);
+// 0: `waves` ranges per resident CTA slot of the GPU (waves >= 1).
+inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_len, int sms,
+                                int split_tokens, int stages_override, bool per_segment,
+                                int waves = 1) {
+  DecodeLaunch L;
+  L.waves = waves < 1 ? 1 : waves;
+  const int G = Hq / Hkv;
+  const int R = q_len * G;
+  L.rows_per_warp = (R <= 4) ? 4 : (R <= 8) ? 8 : 16;  // 4: hi | lo packed MMA columns
+  L.rbg = (R <= 16) ? 1 : (R <= 32 ? 2 : 4);
+  L.rows_per_cta = L.rows_per_warp * L.rbg;
+  L.row_blocks = (R + L.rows_per_cta - 1) / L.rows_per_cta;
+  L.stages = stages_override > 0 ? stages_override : (L.rbg == 1 ? 2 : 3);
+  L.segs = (long long)B * Hkv * L.row_blocks;
+  const long long seg_units = ((long long)max_seq_len + 31) / 32;
+  L.units_max = L.segs * seg_units;
+  L.per_segment = per_segment ? 1 : 0;
+  if (per_segment) {
+    L.grid = L.segs;
+    L.max_units = (int)(seg_units < 1 ? 1 : (seg_units > 0x7FFFFFFF ? 0x7FFFFFFF : seg_units));
+    L.max_portions = 1;
+    L.slots = 0;
+    return L;
+  }
+  long long g;
+  if (split_tokens > 0) {
+    const long long per = (split_tokens + 31) / 32;
+    g = (L.units_max + per - 1) / per;
+  } else {
+    g = (long long)sms * decode_target_occupancy(L.rows_per_warp, L.rbg) * L.waves;
+  }
+  if (g > L.units_max) g = L.units_max;
+  if (g < 1) g = 1;
+  long long mu = (L.units_max + g - 1) / g;
+  if (mu > kMaxUnitsPerCta) {
+    g = (L.units_max + kMaxUnitsPerCta - 1) / kMaxUnitsPerCta;
+    mu = (L.units_max + g - 1) / g;
+  }
+  L.grid = g;
+  L.max_units = (int)(mu < 1 ? 1 : mu);
+  L.max_portions = (int)(L.segs < L.max_units ? L.segs : L.max_units);
+  L.slots = L.segs + g;
+  return L;
+}
+
+// FP8 tensor-core decode kernel.  rows_per_warp is 4, 8 or 16 and rbg (warps that
+// share one K/V stream) 1, 2 or 4; stages 2 or 3.  1-D grid of `grid` CTAs
+// (balanced ranges, or one per segment when p.per_segment).
 cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
-                              cudaStream_t stream);
+                              long long grid, cudaStream_t stream);
+
+// Dynamic shared memory of one decode CTA (rows = min(rows_per_cta, q_len * G)).
+size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units,
+                             int max_portions);
+
+// Balanced mode without a split override: lower L.grid (and raise
+// L.max_units) until the CTAs fill L.waves waves of resident CTAs on `sms`
+// SMs, as far as the shared-memory footprint allows.  Needs a current CUDA device; leaves L alone
+// if the occupancy query fails.
+void decode_fp8_fit_grid(int D, int rows, int sms, DecodeLaunch& L);
 
 // ------------------------------------------------------------ device helpers
 

@@ -19,8 +19,8 @@ struct atlas_kv_pool {
   size_t workspace_bytes;
   int32_t split_override;
   int32_t stages_override;
-  // workspace layout, fixed at creation
-  size_t counters_off, counters_slots, partial_off;
+  int32_t waves_override;
+  size_t counters_bytes;  // largest counter block any accepted call uses
 };
 
 namespace {
@@ -51,57 +51,46 @@ int device_sm_count() {
   return cached[dev];
 }
 
-size_t partial_bytes(int batch, int num_splits, int rows_all, int head_dim) {
-  const size_t lse = align_up((size_t)batch * num_splits * rows_all * sizeof(float), kAlign);
-  const size_t o = align_up((size_t)batch * num_splits * rows_all * head_dim * sizeof(float), kAlign);
-  return lse + o;
+// Workspace of one call: [error word][counters][log2-sum-exp][O partials].
+struct WsLayout {
+  size_t counters, lse, o, total;
+};
+WsLayout ws_layout(const atlas::DecodeLaunch& L, int head_dim) {
+  WsLayout w;
+  w.counters = kAlign;
+  const size_t cnt = align_up((size_t)L.segs * sizeof(int32_t), kAlign);
+  w.lse = w.counters + cnt;
+  const size_t rows = (size_t)L.slots * L.rows_per_cta;
+  w.o = w.lse + align_up(rows * sizeof(float), kAlign);
+  w.total = w.o + align_up(rows * head_dim * sizeof(float), kAlign);
+  return w;
 }
 
-struct Plan {
-  int split_tokens, num_splits, kernel, rows_per_cta, row_blocks, launches, stages;
-  int rows_per_warp, rbg;
-  long long grid_ctas;
-};
-
-// Split-KV partition (A1).  The host sees only max_seq_len, so it sizes the
-// grid as if every sequence were that long; splits past a sequence's end exit
-// at once.  Target one wave of resident CTAs (3 per SM for the 8-row variant,
-// 2 for the 16-row ones), splits a multiple of 64 tokens in [256, kMaxSplit];
-// the chunk adapts to the sequence length and the SM count, the "block size
+// Split-KV partition (A1): balanced ranges of 32-token units, one per resident
+// CTA slot, or ranges of about split_override tokens when one is set.  The
+// range length adapts to the lengths and the SM count -- the "block size
 // adapted to sequence length and architecture" of the Atlas deep-dive's
-// attention paragraph.
-Plan make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len, int max_seq_len,
-               int sms) {
-  Plan pl;
-  const int G = num_q_heads / pool->num_kv_heads;
-  const int R = q_len * G;
-  pl.kernel = 1;
-  // query rows (q_len x group) per warp, and warps sharing one K/V stream
-  pl.rows_per_warp = (R <= 8) ? 8 : 16;
-  pl.rbg = (R <= 16) ? 1 : (R <= 32 ? 2 : 4);
-  pl.rows_per_cta = pl.rows_per_warp * pl.rbg;
-  pl.row_blocks = (R + pl.rows_per_cta - 1) / pl.rows_per_cta;
-  int T;
-  if (pool->split_override > 0) {
-    T = pool->split_override;
-  } else {
-    const long long units = (long long)batch * pool->num_kv_heads * pl.row_blocks;
-    const long long target = (long long)sms * (pl.rows_per_warp == 8 ? 3 : 2);
-    long long want = (target + units - 1) / (units > 0 ? units : 1);
-    if (want < 1) want = 1;
-    long long t = (max_seq_len + want - 1) / want;
-    t = (t + kMinSplit - 1) / kMinSplit * kMinSplit;
-    if (t < 256) t = 256;
-    if (t > kMaxSplit) t = kMaxSplit;
-    T = (int)t;
+// attention paragraph, taken to equal work per CTA.
+atlas::DecodeLaunch make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
+                              int max_seq_len, int sms, bool fit) {
+  atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, pool->num_kv_heads, q_len,
+                                             max_seq_len, sms, pool->split_override,
+                                             pool->stages_override, false,
+                                             pool->waves_override > 0 ? pool->waves_override : 1);
+  if (fit && pool->split_override == 0) {
+    const int R = q_len * (num_q_heads / pool->num_kv_heads);
+    atlas::decode_fp8_fit_grid(pool->head_dim, R < L.rows_per_cta ? R : L.rows_per_cta, sms, L);
   }
-  pl.split_tokens = T;
-  pl.num_splits = (max_seq_len + T - 1) / T;
-  if (pl.num_splits < 1) pl.num_splits = 1;
-  pl.launches = 1;
-  pl.stages = pool->stages_override > 0 ? pool->stages_override : (pl.rbg == 1 ? 2 : 3);
-  pl.grid_ctas = (long long)pl.num_splits * pl.row_blocks * pool->num_kv_heads * batch;
-  return pl;
+  return L;
+}
+
+bool device_present() {
+  int cnt = 0;
+  if (cudaGetDeviceCount(&cnt) != cudaSuccess || cnt <= 0) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
 }
 
 }  // namespace
@@ -123,14 +112,26 @@ const char* atlas_status_string(atlas_status_t s) {
 }
 
 size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t num_q_heads,
-                                int32_t head_dim, int32_t max_seq_len, int32_t min_split_tokens) {
-  if (max_batch < 0 || max_q_len < 1 || num_q_heads < 1 || max_seq_len < 0) return 0;
+                                int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
+                                int32_t min_split_tokens) {
+  if (max_batch < 0 || max_q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || max_seq_len < 0)
+    return 0;
+  if (num_q_heads % num_kv_heads != 0) return 0;
   if (head_dim != 64 && head_dim != 128) return 0;
-  if (min_split_tokens <= 0) min_split_tokens = kMinSplit;
-  const int max_splits = (max_seq_len + min_split_tokens - 1) / min_split_tokens;
-  const size_t counters = align_up((size_t)max_batch * num_q_heads * max_q_len * sizeof(int32_t), kAlign);
-  return kAlign + counters +
-         partial_bytes(max_batch, max_splits > 0 ? max_splits : 1, max_q_len * num_q_heads, head_dim);
+  if (min_split_tokens < 0) return 0;
+  const int sms = device_present() ? device_sm_count() : kDefaultSms;
+  size_t need = 0;
+  for (int ql = 1; ql <= max_q_len; ++ql) {
+    const int msl = max_seq_len > ql ? max_seq_len : ql;
+    // the automatic plan, and the finest split override the caller will set
+    for (int split : {0, min_split_tokens}) {
+      const atlas::DecodeLaunch L =
+          atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, msl, sms, split, 0, false);
+      const size_t t = ws_layout(L, head_dim).total;
+      if (t > need) need = t;
+    }
+  }
+  return need;
 }
 
 atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, int32_t page_size,
@@ -148,8 +149,13 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   if (!k_pages || !v_pages || !k_scale || !v_scale || !workspace) return ATLAS_ERR_INVALID_ARG;
   if (!aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(workspace, kAlign))
     return ATLAS_ERR_INVALID_ARG;
-  const size_t counters_slots = (size_t)max_batch * num_q_heads * max_q_len;
-  const size_t counters_bytes = align_up(counters_slots * sizeof(int32_t), kAlign);
+  size_t counters_bytes = 0;
+  for (int ql = 1; ql <= max_q_len; ++ql) {
+    const atlas::DecodeLaunch L = atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, ql,
+                                                     kDefaultSms, 0, 0, false);
+    const size_t c = align_up((size_t)L.segs * sizeof(int32_t), kAlign);
+    if (c > counters_bytes) counters_bytes = c;
+  }
   if (workspace_bytes < kAlign + counters_bytes) return ATLAS_ERR_WORKSPACE;
   atlas_kv_pool* p = new (std::nothrow) atlas_kv_pool;
   if (!p) return ATLAS_ERR_INVALID_ARG;
@@ -168,9 +174,8 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   p->workspace_bytes = workspace_bytes;
   p->split_override = 0;
   p->stages_override = 0;
-  p->counters_off = kAlign;
-  p->counters_slots = counters_slots;
-  p->partial_off = kAlign + counters_bytes;
+  p->waves_override = 0;
+  p->counters_bytes = counters_bytes;
   *out = p;
   return ATLAS_OK;
 }
@@ -197,6 +202,10 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
     case ATLAS_OPT_STAGES:
       if (value != 0 && value != 2 && value != 3) return ATLAS_ERR_INVALID_ARG;
       pool->stages_override = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_WAVES:
+      if (value < 0 || value > 8) return ATLAS_ERR_INVALID_ARG;
+      pool->waves_override = value;
       return ATLAS_OK;
   }
   return ATLAS_ERR_INVALID_ARG;
@@ -251,18 +260,16 @@ atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t 
   atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
   if (st != ATLAS_OK) return st;
   if (!plan || n < 0) return ATLAS_ERR_INVALID_ARG;
-  int sms = kDefaultSms;
-  {
-    int dev = 0, cnt = 0;
-    if (cudaGetDeviceCount(&cnt) == cudaSuccess && cnt > 0 && cudaGetDevice(&dev) == cudaSuccess)
-      sms = device_sm_count();
-    else
-      cudaGetLastError();
-  }
-  const Plan pl = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms);
-  const int32_t f[ATLAS_PLAN_FIELDS] = {pl.split_tokens, pl.num_splits, pl.kernel,
-                                        pl.rows_per_cta, pl.row_blocks, pl.launches,
-                                        (int32_t)(pl.grid_ctas > 0x7FFFFFFF ? 0x7FFFFFFF : pl.grid_ctas)};
+  const bool dev = device_present();
+  const int sms = dev ? device_sm_count() : kDefaultSms;
+  const atlas::DecodeLaunch L = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, dev);
+  const long long seg_units = ((long long)max_seq_len + 31) / 32;
+  long long spread = 1 + (seg_units - 1 + L.max_units - 1) / L.max_units;
+  if (spread > L.grid) spread = L.grid;
+  const int32_t split = pool->split_override > 0 ? pool->split_override : 32 * L.max_units;
+  const int32_t f[ATLAS_PLAN_FIELDS] = {split, (int32_t)spread, 1, L.rows_per_cta,
+                                        L.row_blocks, 1,
+                                        (int32_t)(L.grid > 0x7FFFFFFF ? 0x7FFFFFFF : L.grid)};
   for (int i = 0; i < n && i < ATLAS_PLAN_FIELDS; ++i) plan[i] = f[i];
   return ATLAS_OK;
 }
@@ -290,15 +297,10 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
     return ATLAS_ERR_INVALID_ARG;
 
   const int sms = device_sm_count();
-  const Plan pl = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms);
-  const int rows_all = q_len * num_q_heads;
-  if ((size_t)batch * pool->num_kv_heads * pl.row_blocks > pool->counters_slots)
-    return ATLAS_ERR_WORKSPACE;
-  if (pl.num_splits > 1 &&
-      pool->partial_off + partial_bytes(batch, pl.num_splits, rows_all, pool->head_dim) >
-          pool->workspace_bytes)
-    return ATLAS_ERR_WORKSPACE;
-  if (pl.num_splits > 65535 * 16 || batch > 65535) return ATLAS_ERR_UNSUPPORTED;
+  const atlas::DecodeLaunch L = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true);
+  const WsLayout ws = ws_layout(L, pool->head_dim);
+  if (ws.total > pool->workspace_bytes) return ATLAS_ERR_WORKSPACE;
+  if (L.grid > 0x7FFFFFFFLL) return ATLAS_ERR_UNSUPPORTED;
 
   atlas::DecodeParams p{};  // value-initialised: no fused append unless set
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -309,13 +311,11 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.out = static_cast<__nv_bfloat16*>(out);
-  uint8_t* ws = pool->workspace;
-  p.err = reinterpret_cast<int32_t*>(ws);
-  p.counters = reinterpret_cast<int32_t*>(ws + pool->counters_off);
-  const size_t lse_bytes =
-      align_up((size_t)batch * pl.num_splits * rows_all * sizeof(float), kAlign);
-  p.part_lse = reinterpret_cast<float*>(ws + pool->partial_off);
-  p.part_o = reinterpret_cast<float*>(ws + pool->partial_off + lse_bytes);
+  uint8_t* wsp = pool->workspace;
+  p.err = reinterpret_cast<int32_t*>(wsp);
+  p.counters = reinterpret_cast<int32_t*>(wsp + ws.counters);
+  p.part_lse = reinterpret_cast<float*>(wsp + ws.lse);
+  p.part_o = reinterpret_cast<float*>(wsp + ws.o);
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = pool->num_kv_heads;
@@ -325,15 +325,17 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.ps = pool->page_size;
   p.num_pages = pool->num_pages;
   p.max_blocks = max_blocks_per_seq;
-  p.split_tokens = pl.split_tokens;
-  p.num_splits = pl.num_splits;
-  p.row_blocks = pl.row_blocks;
+  p.max_seq_len = max_seq_len;
+  p.row_blocks = L.row_blocks;
+  p.max_units = L.max_units;
+  p.max_portions = L.max_portions;
+  p.per_segment = 0;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)pool->head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
   p.k_new = k_new;
   p.v_new = v_new;
   p.new_dtype = new_dtype;
-  cudaError_t e = atlas::launch_decode_fp8(p, pl.rows_per_warp, pl.rbg, pl.stages,
+  cudaError_t e = atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
@@ -377,7 +379,10 @@ atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream,
           cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return ATLAS_ERR_CUDA;
-  if (host != 0 && (cudaMemsetAsync(pool->workspace, 0, sizeof(int32_t), s) != cudaSuccess ||
+  // a call that stopped early (a timed-out wait) can leave completion counters
+  // set: clear them with the error word
+  if (host != 0 && (cudaMemsetAsync(pool->workspace, 0, kAlign + pool->counters_bytes, s) !=
+                        cudaSuccess ||
                     cudaStreamSynchronize(s) != cudaSuccess))
     return ATLAS_ERR_CUDA;
   *code = host;

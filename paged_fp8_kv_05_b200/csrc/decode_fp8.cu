@@ -22,11 +22,11 @@
 // A bf16 significand has 8 bits, hi keeps 4 and lo the next 4, so the pair is
 // exact unless lo falls below the E4M3 normal range (a contribution under
 // 2^-9 of the row's largest element).  The probabilities are taken as
-// p = 2^(s - m + 8) in f32 (so 2^-6 <= p <= 2^8 covers the useful range),
-// rounded to f16 and split the same way (hi + lo carries 8 significant bits).
-// The row sum l accumulates the f32 p, and out = O / l, so the 2^8 and a_r
-// factors cancel exactly.  Error budget: the 8-bit P adds ~1e-4 relative L2 to
-// the bf16 output rounding (~1.7e-3) on the benchmark workloads.
+// p = 2^(s - m + 8) in f32, rounded to f16 and split the same way (hi + lo
+// carries 8 significant bits).  The row sum l accumulates the f32 p, and
+// out = O / l, so the 2^8 and a_r factors cancel exactly.  The 8-bit P adds
+// ~1e-4 relative L2 to the bf16 output rounding (~1.7e-3) on the benchmark
+// workloads.
 //
 // Fragment layouts.  The head dimension is permuted consistently between K and
 // Q: k-step s = 2j + hs of 32 dims reads bytes 64j + 16c + 8hs + {0..7} of a
@@ -38,21 +38,28 @@
 // accumulator through movmatrix.trans, which hands each lane exactly those
 // four tokens of its row -- no shuffles.
 //
-// Work split and staging.  CTA (split s, KV head h, sequence b, row group)
-// owns the KV tokens [s*T, min((s+1)*T, L_b)) and RBG blocks of 8*NT query rows.
-// Its 4 warps form 4/RBG streams; the RBG warps of a stream share one ring of S
-// shared-memory stages, each holding the K tiles and V^T tiles of one 32-token
-// unit (two 16-token page pieces, each a contiguous block of 16*D bytes in its
-// page), filled by 1-D bulk copies (cp.async.bulk, no multicast) completing
-// on a "full" mbarrier; with RBG > 1 an "empty" mbarrier counts the
-// consumers before a stage is refilled.  Streams take units round-robin with
-// private online-softmax state and are combined in shared memory.  A sequence
-// with one split writes bf16 output directly; otherwise each split writes
-// (O/l, log2-sum-exp) to the workspace and the CTA that finishes a
-// (b, h, row group) last -- one atomic counter, no waiting -- merges the splits
-// and resets the counter.  Every mbarrier wait is bounded (200 ms of wall
-// clock): a wait that runs out flags ATLAS_DEVERR_TIMEOUT and the warp stops
-// computing after draining the loads it issued.
+// Work partition (persistent, balanced).  A segment is (sequence b, KV head h,
+// row group rg): ceil(L_b / 32) units of 32 KV tokens for up to RC query rows.
+// All units of all segments form one list (segments in (b, h, rg) order);
+// CTA c of the G CTAs takes units [c*U/G, (c+1)*U/G) of the U in the list, so
+// every CTA gets the same amount of KV to stream whatever the length mix (the
+// "block size adapted to sequence length" of the deep-dive, taken to its
+// limit).  Its range cuts the list into portions, one per segment it touches.
+// Its 4 warps form 4/RBG streams that take the CTA's units round-robin; the RBG
+// warps of a stream share one ring of S shared-memory stages, each holding the
+// K and V^T pieces of one unit (two 16-token page pieces, each a contiguous
+// block of 16*D bytes in its page), filled by 1-D bulk copies (cp.async.bulk,
+// no multicast) that complete on a "full" mbarrier; with RBG > 1 an "empty"
+// mbarrier counts the consumers before a stage is refilled.  The ring keeps
+// streaming across portion boundaries.  At the end of a portion the streams
+// combine their online-softmax states in shared memory; a segment that lies
+// inside one CTA is written out as bf16, otherwise the CTA writes
+// (O/l, log2-sum-exp) to the partial slot (segment + c) and the CTA that
+// finishes the segment last -- one atomic counter per segment, no waiting --
+// merges its slots and resets the counter.  A per-segment mode (CTA c = segment
+// c, no partials) serves callers with little scratch.  Every mbarrier wait is
+// bounded (200 ms of wall clock): a wait that runs out flags
+// ATLAS_DEVERR_TIMEOUT and the warp stops computing after draining its loads.
 #include <float.h>
 #include <math.h>
 
@@ -65,7 +72,8 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
-constexpr int kUnit = 32;  // tokens per pipeline unit (two 16-token tiles)
+constexpr int kUnit = 32;  // tokens per pipeline unit (two 16-token pieces)
+constexpr int kQBuf = 3;   // Q row buffers: portion pi + 2 loads while pi computes
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -133,153 +141,348 @@ __device__ __forceinline__ uint32_t token_mask4(int nvalid, int c) {
          (2 * c + 8 < nvalid ? 0x00FF0000u : 0u) | (2 * c + 9 < nvalid ? 0xFF000000u : 0u);
 }
 
+// 16-byte global -> shared copy that completes asynchronously (cp.async, L2 only)
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_group1() {  // all but the newest group
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 // ----------------------------------------------------------- shared memory plan
 
-template <int D, int S, int NSTREAM, int RC>
-struct Smem {
-  static constexpr int TILE = 16 * D;     // one 16-token K tile or V^T tile
-  static constexpr int STAGE = 4 * TILE;  // K_A, K_B, V_A, V_B
-  static constexpr size_t RING = (size_t)NSTREAM * S * STAGE;
-  // stream-combine buffers (m, l, O) reuse the ring after the main loop
-  static constexpr size_t COMBINE = NSTREAM > 1 ? (size_t)NSTREAM * RC * (D + 2) * 4 : 0;
-  static constexpr size_t REGION = RING > COMBINE ? RING : (COMBINE + 1023) / 1024 * 1024;
-  static constexpr size_t BARS = REGION;                            // full[], empty[]
-  static constexpr size_t PIDS = BARS + (size_t)2 * NSTREAM * S * 8;
-  static size_t total(int split_tokens) { return PIDS + (size_t)(split_tokens / 16 + 2) * 4 + 1024; }
+// One portion: the part of segment (b, seg) that lies in this CTA's range.
+struct Portion {
+  int b, seg;           // sequence, segment within the sequence (h * row_blocks + rg)
+  int L;                // the sequence's length
+  int ua;               // first unit of the portion inside the segment
+  int k0;               // first unit of the portion inside the CTA's range
+  int c_first, c_last;  // first and last CTA that hold part of the segment
+  float k_scale, v_scale;  // the KV head's dequantisation scales
 };
+
+// Dynamic shared memory: [ring][mbarriers][Q rows x kQBuf][combine][unit pieces]
+// [portions].  Only 16-byte alignment is needed (bulk copies, cp.async,
+// ldmatrix, vector loads).
+struct SmemPlan {
+  size_t bars, qbuf, combine, pieces, portions, total;
+};
+__host__ __device__ inline SmemPlan smem_plan(int D, int S, int nstream, int rows, int max_units,
+                                              int max_portions) {
+  SmemPlan sp;
+  const size_t ring = (size_t)nstream * S * 4 * 16 * D;
+  sp.bars = ring;
+  sp.qbuf = sp.bars + (size_t)2 * nstream * S * 8;
+  sp.combine = sp.qbuf + (size_t)kQBuf * rows * D * 2;
+  // per stream and row: m and l (float), O / l (half)
+  const size_t comb = nstream > 1 ? (size_t)nstream * rows * (8 + 2 * D) : 0;
+  sp.pieces = sp.combine + (comb + 15) / 16 * 16;
+  sp.portions = sp.pieces + (size_t)max_units * 8;
+  sp.total = sp.portions + (size_t)max_portions * sizeof(Portion) + 16;
+  return sp;
+}
+
+// Exclusive prefix sum of v over the CTA's threads (all threads call it);
+// `total` receives the sum over the CTA.  `warp_sums` holds kWarps entries.
+__device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long long v,
+                                                                  unsigned long long* warp_sums,
+                                                                  unsigned long long& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  unsigned long long base = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) base += warp_sums[w];
+    total += warp_sums[w];
+  }
+  __syncthreads();  // warp_sums may be reused
+  return base + incl - v;
+}
+
+// CTA that owns global unit u under the balanced partition of U units over G CTAs
+__device__ __forceinline__ int owner_cta(long long u, long long U, int G) {
+  return (int)(((u + 1) * G - 1) / U);
+}
 
 // ------------------------------------------------------------------- the kernel
 
-template <int D, int NT, int RBG, int S>
+template <int D, int NT, int RBG, int S, bool PK>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     paged_decode_fp8_kernel(const DecodeParams p) {
-  constexpr int RW = 8 * NT;             // query rows per warp
+  // PK (packed): a warp holds 4 query rows, and the 8 columns of every MMA's N
+  // side carry the hi parts (columns 0-3) and the lo parts (columns 4-7) of
+  // those rows' Q (for QK^T) and P (for PV), so one MMA does the work of two
+  static_assert(!PK || (NT == 1 && RBG == 1), "packed mode is 4 rows, one warp per stream");
+  constexpr int RW = PK ? 4 : 8 * NT;    // query rows per warp
   constexpr int RC = RW * RBG;           // query rows per CTA
   constexpr int NSTREAM = kWarps / RBG;  // unit streams per CTA
   constexpr int NCH = D / 64;            // 16-byte K chunks per token per lane
   constexpr int KSTEP = D / 32;          // k-steps of QK^T
   constexpr int MT = D / 16;             // m-tiles of O^T
-  using SM = Smem<D, S, NSTREAM, RC>;
-  constexpr int TILE = SM::TILE;
-  constexpr int STAGE = SM::STAGE;
+  constexpr int TILE = 16 * D;           // one 16-token K piece or V^T piece
+  constexpr int STAGE = 4 * TILE;        // K_A, K_B, V_A, V_B
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int Rtot = p.q_len * p.G;
+  const int rows_max = min(RC, Rtot);    // rows of the fullest row group
+  extern __shared__ __align__(16) uint8_t smem[];
+  const SmemPlan sp = smem_plan(D, S, NSTREAM, rows_max, p.max_units, p.max_portions);
   uint8_t* ring = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + SM::BARS);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty_bar = full_bar + NSTREAM * S;
-  int* s_piece = reinterpret_cast<int*>(smem + SM::PIDS);
+  __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(smem + sp.qbuf);
+  float* s_cm = reinterpret_cast<float*>(smem + sp.combine);  // [NSTREAM][rows_max]
+  float* s_cl = s_cm + NSTREAM * rows_max;                      // [NSTREAM][rows_max]
+  __half* s_co = reinterpret_cast<__half*>(s_cl + NSTREAM * rows_max);  // [NSTREAM][rows_max][D]
+  int2* s_pieces = reinterpret_cast<int2*>(smem + sp.pieces);
+  Portion* s_port = reinterpret_cast<Portion*>(smem + sp.portions);
   __shared__ int s_is_last;
+  __shared__ int s_nport;
+  __shared__ unsigned long long s_scan[kWarps];
+  __shared__ float s_rowM[RC], s_rowD[RC];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, c = lane & 3;
   const int stream = warp / RBG, rbw = warp % RBG;
-  const int n_groups = p.row_blocks;  // row groups of RC rows per (b, h)
-  const int grp = blockIdx.x % n_groups;
-  const int split = blockIdx.x / n_groups;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int L = __ldg(p.seq_lens + b);
-  const int Rtot = p.q_len * p.G;
-  const int cta_row0 = grp * RC;
-  const int rows_cta = min(RC, Rtot - cta_row0);
-  const int row0 = cta_row0 + rbw * RW;  // this warp's first row
+  const int cid = blockIdx.x, G = gridDim.x;
+  const int RB = p.row_blocks;          // row groups per (b, h)
+  const int Hs = p.Hkv * RB;            // segments per sequence
+  auto valid_len = [&](int L) {
+    return L >= p.q_len && L <= p.max_blocks * p.ps && L <= p.max_seq_len;
+  };
+  auto units_of = [&](int L) { return (L + kUnit - 1) / kUnit; };
 
-  // ---- invalid sequence: zero this CTA's rows once (split 0) and flag it
-  if (L < p.q_len || L > p.max_blocks * p.ps || L > p.num_splits * p.split_tokens) {
-    if (split == 0) {
+  // ---- invalid sequences (shorter than q_len, longer than the block-table row
+  // or the host's max_seq_len): zero all their rows and flag them; one CTA per b
+  for (int bb = cid; bb < p.B; bb += G) {
+    const int L = __ldg(p.seq_lens + bb);
+    if (valid_len(L)) continue;
+    if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
+    const size_t n = (size_t)p.q_len * p.Hq * D;
+    __nv_bfloat16* o = p.out + (size_t)bb * n;
+    for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
+  }
+
+  // ---- this CTA's range of units and its portions (A1)
+  long long u0 = 0, u1 = 0;
+  if (p.per_segment) {
+    // CTA cid is segment cid: the whole segment, one portion, no partial
+    const int b = cid / Hs, seg = cid % Hs;
+    const int L = __ldg(p.seq_lens + b);
+    if (!valid_len(L)) return;  // CTA-uniform
+    if (tid == 0) {
+      Portion P;
+      P.b = b; P.seg = seg; P.L = L; P.ua = 0; P.k0 = 0; P.c_first = P.c_last = cid;
+      P.k_scale = __ldg(p.k_scale + seg / RB);
+      P.v_scale = __ldg(p.v_scale + seg / RB);
+      s_port[0] = P;
+      s_nport = 1;
+    }
+    u1 = units_of(L);
+  } else {
+    // every thread takes a contiguous run of sequences; a block-wide exclusive
+    // scan of the runs' unit counts gives each run's first global unit
+    const int per = (p.B + kThreads - 1) / kThreads;
+    const int bb0 = min(p.B, tid * per), bb1 = min(p.B, bb0 + per);
+    unsigned long long mine = 0;
+    for (int bb = bb0; bb < bb1; ++bb) {
+      const int L = __ldg(p.seq_lens + bb);
+      if (valid_len(L)) mine += (unsigned long long)Hs * units_of(L);
+    }
+    unsigned long long total = 0;
+    const unsigned long long first = block_exclusive_scan(mine, s_scan, total);
+    const long long U = (long long)total;
+    // with fewer units than CTAs only the first U CTAs take one unit each, so
+    // that every CTA between the first and last owner of a segment holds part
+    // of it (the merge counts on that)
+    const int Ge = (int)min((long long)G, U);
+    if (cid >= Ge) return;  // CTA-uniform from here on (U == 0 included)
+    u0 = (long long)((unsigned long long)cid * total / Ge);
+    u1 = (long long)((unsigned long long)(cid + 1) * total / Ge);
+    if (u1 - u0 > p.max_units) {  // only if a length exceeded the host's bound
       if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
-      for (int idx = tid; idx < rows_cta * D; idx += kThreads) {
-        const int r = cta_row0 + idx / D, d = idx % D;
-        const int i = r / p.G, hq = h * p.G + r % p.G;
-        p.out[(((size_t)b * p.q_len + i) * p.Hq + hq) * D + d] = __float2bfloat16_rn(0.f);
+      return;
+    }
+    // portions: the segments of this thread's sequences that meet [u0, u1),
+    // counted, scanned and written in list order (no sorting needed)
+    int n_mine = 0;
+    {
+      long long P = (long long)first;
+      for (int bb = bb0; bb < bb1 && P < u1; ++bb) {
+        const int L = __ldg(p.seq_lens + bb);
+        if (!valid_len(L)) continue;
+        const int n = units_of(L);
+        const long long size = (long long)Hs * n;
+        if (P + size > u0) {
+          const long long s_lo = max(u0 - P, 0LL) / n;
+          const long long s_hi = (min(u1, P + size) - 1 - P) / n;
+          n_mine += (int)(s_hi - s_lo + 1);
+        }
+        P += size;
       }
     }
-    return;
+    unsigned long long n_all = 0;
+    int slot_out = (int)block_exclusive_scan((unsigned long long)n_mine, s_scan, n_all);
+    if (tid == 0) s_nport = (int)n_all;
+    {
+      long long P = (long long)first;
+      for (int bb = bb0; bb < bb1 && P < u1; ++bb) {
+        const int L = __ldg(p.seq_lens + bb);
+        if (!valid_len(L)) continue;
+        const int n = units_of(L);
+        const long long size = (long long)Hs * n;
+        if (P + size > u0) {
+          const int s_lo = (int)(max(u0 - P, 0LL) / n);
+          const int s_hi = (int)((min(u1, P + size) - 1 - P) / n);
+          for (int seg = s_lo; seg <= s_hi; ++seg) {
+            const long long s0 = P + (long long)seg * n;
+            const long long a = max(s0, u0);
+            Portion Q;
+            Q.b = bb; Q.seg = seg; Q.L = L;
+            Q.ua = (int)(a - s0);
+            Q.k0 = (int)(a - u0);
+            Q.c_first = owner_cta(s0, U, Ge);
+            Q.c_last = owner_cta(s0 + n - 1, U, Ge);
+            Q.k_scale = __ldg(p.k_scale + seg / RB);
+            Q.v_scale = __ldg(p.v_scale + seg / RB);
+            s_port[slot_out++] = Q;
+          }
+        }
+        P += size;
+      }
+    }
   }
-  const int t_begin = split * p.split_tokens;
-  if (t_begin >= L) return;
-  const int t_end = min(t_begin + p.split_tokens, L);
-  const int n_split_b = (L + p.split_tokens - 1) / p.split_tokens;
+  __syncthreads();
+  const int n_port = s_nport;
+  const int U_cta = (int)(u1 - u0);
+  // portion p covers CTA units [k0_p, k0_{p+1})
+  auto port_end = [&](int pi) { return pi + 1 < n_port ? s_port[pi + 1].k0 : U_cta; };
 
-  // ---- A0, fused append: quantise and store the step's new tokens that fall in
-  // this split (positions L - q_len .. L - 1), then order those global writes
-  // before the bulk copies that read the pages back
+  // Q rows of portion pi -> Q buffer pi % kQBuf, one cp.async group per call
+  auto prefetch_q = [&](int pi) {
+    const Portion P = s_port[pi];
+    const int h = P.seg / RB, r0 = (P.seg % RB) * RC;
+    const int rows = min(RC, Rtot - r0);
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    __nv_bfloat16* dst = s_q + (size_t)(pi % kQBuf) * rows_max * D;
+    for (int idx = tid; idx < rows * CPR; idx += kThreads) {
+      const int lr = idx / CPR, ch = idx - lr * CPR;
+      const int r = r0 + lr;
+      const int i = r / p.G, hq = h * p.G + r % p.G;
+      cp_async16(dst + lr * D + ch * 8,
+                 p.q + (((size_t)P.b * p.q_len + i) * p.Hq + hq) * D + ch * 8);
+    }
+    cp_async_commit();
+  };
+  prefetch_q(0);
+  if (n_port > 1) prefetch_q(1);
+
+  // ---- A2, block-table gather: the two 16-token pieces of unit k of the
+  // range, as indices of 16*D-byte blocks of the page arrays (-1: past the end
+  // of the sequence or a bad page id).  The divisions happen here, once.
+  const int groups_per_page = p.ps / 16;
+  auto build_piece = [&](int k) {
+    int lo = 0, hi = n_port - 1;   // last portion with k0 <= k
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_port[mid].k0 <= k) lo = mid; else hi = mid - 1;
+    }
+    const Portion P = s_port[lo];
+    const int h = P.seg / RB;
+    const int t0 = kUnit * (P.ua + k - P.k0);
+    int pc[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int t = t0 + 16 * half;
+      pc[half] = -1;
+      if (t < P.L) {
+        const int pg = t / p.ps;
+        const int pid = __ldg(p.block_table + (size_t)P.b * p.max_blocks + pg);
+        if (pid < 0 || pid >= p.num_pages)
+          atomicOr(p.err, ATLAS_DEVERR_PAGE_ID);
+        else
+          pc[half] = (pid * p.Hkv + h) * groups_per_page + (t - pg * p.ps) / 16;
+      }
+    }
+    s_pieces[k] = make_int2(pc[0], pc[1]);
+  };
+  // ---- A0, fused append: the step's new tokens (positions L - q_len .. L - 1)
+  // that fall in this CTA's portions are quantised and stored first, while HBM
+  // is still idle, and made visible to the bulk copies before any is queued
   if (p.k_new != nullptr) {
-    const int first_new = L - p.q_len;
-    const int a0 = max(t_begin, first_new);
-    const int n_tok = t_end - a0;
-    if (n_tok > 0) {
+    bool wrote = false;
+    for (int pi = 0; pi < n_port; ++pi) {
+      const Portion P = s_port[pi];
+      const int L = P.L;
+      const int h = P.seg / RB;
+      const int first_new_pos = L - p.q_len;
+      const int a0 = max(kUnit * P.ua, first_new_pos);
+      const int a1 = min(kUnit * (P.ua + port_end(pi) - P.k0), L);
+      const int n_tok = a1 - a0;
+      if (n_tok <= 0) continue;
+      wrote = true;
       constexpr int CH = D / 16;
       for (int idx = tid; idx < 2 * n_tok * CH; idx += kThreads) {
         const int which = idx / (n_tok * CH);  // 0 = K, 1 = V
         const int r = idx - which * n_tok * CH;
         const int pos = a0 + r / CH, j = r % CH;
-        const int page = __ldg(p.block_table + (size_t)b * p.max_blocks + pos / p.ps);
+        const int page = __ldg(p.block_table + (size_t)P.b * p.max_blocks + pos / p.ps);
         if (page < 0 || page >= p.num_pages) {
           atomicOr(p.err, ATLAS_DEVERR_APPEND);
           continue;
         }
         float x[16];
         load16_as_f32(which ? p.v_new : p.k_new,
-                      (((size_t)b * p.q_len + (pos - first_new)) * p.Hkv + h) * D + 16 * j,
+                      (((size_t)P.b * p.q_len + (pos - first_new_pos)) * p.Hkv + h) * D + 16 * j,
                       p.new_dtype, x);
-        const uint4 codes = quantize16_e4m3(x, __ldg((which ? p.v_scale : p.k_scale) + h));
+        const uint4 codes = quantize16_e4m3(x, which ? P.v_scale : P.k_scale);
         const size_t head_page = (size_t)page * p.Hkv + h;
         if (!which)
           store16_k(const_cast<uint8_t*>(p.k_pages), head_page, D, p.ps, pos % p.ps, j, codes);
         else
           store16_v(const_cast<uint8_t*>(p.v_pages), head_page, D, p.ps, pos % p.ps, j, codes);
       }
+    }
+    if (wrote) {
       __threadfence();
       fence_proxy_async_global();
     }
   }
-
-  // ---- A2, block-table gather: index of every 16-token piece of this split,
-  // counted in 16*D-byte blocks of the page arrays (-1 for a bad page id).
-  // Piece k holds tokens [t_begin + 16k, +16): page (t / ps), slot group
-  // (t % ps) / 16; the divisions happen here once, not per unit.
-  const int n_pieces = (t_end - t_begin + 15) / 16;
-  const int groups_per_page = p.ps / 16;
-  for (int k = tid; k < n_pieces; k += kThreads) {
-    const int t = t_begin + 16 * k;
-    const int pg = t / p.ps;
-    int pid = __ldg(p.block_table + (size_t)b * p.max_blocks + pg);
-    int piece = -1;
-    if (pid < 0 || pid >= p.num_pages) {
-      atomicOr(p.err, ATLAS_DEVERR_PAGE_ID);
-    } else {
-      piece = (pid * p.Hkv + h) * groups_per_page + (t - pg * p.ps) / 16;
-    }
-    s_piece[k] = piece;
-  }
+  // the whole unit table, before any bulk copy is queued
+  for (int k = tid; k < U_cta; k += kThreads) build_piece(k);
   if (tid < NSTREAM * S) {
     mbar_init(&full_bar[tid], 1);
     mbar_init(&empty_bar[tid], RBG);
   }
   if (tid == 0) fence_mbar_init();
+  __syncthreads();  // table, barriers and appended tokens ready
 
-  __syncthreads();  // page ids and barrier init visible
-
-  // this stream's units: u = stream + NSTREAM * i, i < n_my
-  const int n_units = (t_end - t_begin + kUnit - 1) / kUnit;
-  const int n_my = (stream < n_units) ? (n_units - stream + NSTREAM - 1) / NSTREAM : 0;
+  // this stream's units: k = stream + NSTREAM * i, i < n_my
+  const int n_my = (stream < U_cta) ? (U_cta - stream + NSTREAM - 1) / NSTREAM : 0;
   const bool producer = (rbw == 0) && (lane == 0);
-  auto unit_t0 = [&](int i) { return t_begin + kUnit * (stream + NSTREAM * i); };
-  // pieces of unit i: 2(stream + NSTREAM i) and the next one (if inside the split)
-  auto piece_of = [&](int k) { return k < n_pieces ? s_piece[k] : -1; };
-
   constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
   auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
     const int st = i % S;
-    const int k = 2 * (stream + NSTREAM * i);
     uint64_t* bar = &full_bar[stream * S + st];
     uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
-    const int pa = piece_of(k), pb = piece_of(k + 1);
-    const uint32_t bytes = (pa >= 0 ? 2 * TILE : 0) + (pb >= 0 ? 2 * TILE : 0);
+    const int2 pc = s_pieces[stream + NSTREAM * i];
+    const uint32_t bytes = (pc.x >= 0 ? 2 * TILE : 0) + (pc.y >= 0 ? 2 * TILE : 0);
     if (bytes == 0) {
       mbar_arrive(bar);
       return;
@@ -287,115 +490,27 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     mbar_arrive_expect_tx(bar, bytes);
     // a 16-token piece is TILE contiguous bytes in both layouts: K rows
     // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
-    if (pa >= 0) {
-      bulk_load(dst, p.k_pages + (size_t)pa * kPiece, TILE, bar);
-      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pa * kPiece, TILE, bar);
+    if (pc.x >= 0) {
+      bulk_load(dst, p.k_pages + (size_t)pc.x * kPiece, TILE, bar);
+      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pc.x * kPiece, TILE, bar);
     }
-    if (pb >= 0) {
-      bulk_load(dst + TILE, p.k_pages + (size_t)pb * kPiece, TILE, bar);
-      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pb * kPiece, TILE, bar);
+    if (pc.y >= 0) {
+      bulk_load(dst + TILE, p.k_pages + (size_t)pc.y * kPiece, TILE, bar);
+      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pc.y * kPiece, TILE, bar);
     }
   };
-
-
-  // the first S units of every stream go out before the query is prepared,
-  // so their loads overlap the Q fetch and split below
   if (producer) {
     for (int i = 0; i < S && i < n_my; ++i) issue(i);
   }
 
-  // ---- Q^T fragments as E4M3 hi + lo with a per-row power-of-two scale
-  // B operand of k-step s = 2j + hs: b0 = dims 64j+16c+8hs+{0..3}, b1 = +{4..7}.
-  uint32_t qhi[NT][KSTEP][2], qlo[NT][KSTEP][2];
-  float alpha_row[NT];  // the scale of row 8nt + g8
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int r = row0 + 8 * nt + g8;
-    float x[NCH][16];
-    if (r < Rtot) {
-      const int i = r / p.G, hq = h * p.G + r % p.G;
-      const __nv_bfloat16* qrow = p.q + (((size_t)b * p.q_len + i) * p.Hq + hq) * D;
-#pragma unroll
-      for (int j = 0; j < NCH; ++j) {
-        const uint4* src = reinterpret_cast<const uint4*>(qrow + j * 64 + 16 * c);
-        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-        const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          x[j][2 * k] = __uint_as_float(wv[k] << 16);
-          x[j][2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < NCH; ++j)
-#pragma unroll
-        for (int k = 0; k < 16; ++k) x[j][k] = 0.f;
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int j = 0; j < NCH; ++j)
-#pragma unroll
-      for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[j][k]));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-    // a = 2^(135 - e) puts amax in [256, 512); halve it if amax * a > 448
-    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF);
-    float a = 1.f;
-    if (amax > 0.f) {
-      const int ex = min(254, max(1, 262 - e));
-      a = __uint_as_float((uint32_t)ex << 23);
-      if (amax * a > 448.f) a *= 0.5f;
-    }
-    alpha_row[nt] = a;
-#pragma unroll
-    for (int j = 0; j < NCH; ++j)
-#pragma unroll
-      for (int hs = 0; hs < 2; ++hs)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int k0 = 8 * hs + 4 * half;
-          const float y0 = x[j][k0] * a, y1 = x[j][k0 + 1] * a;
-          const float y2 = x[j][k0 + 2] * a, y3 = x[j][k0 + 3] * a;
-          const uint32_t h01 = f32x2_to_e4m3x2(y0, y1), h23 = f32x2_to_e4m3x2(y2, y3);
-          const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
-          const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
-          const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
-          const uint32_t l01 = f32x2_to_e4m3x2(y0 - b01.x, y1 - b01.y);
-          const uint32_t l23 = f32x2_to_e4m3x2(y2 - b23.x, y3 - b23.y);
-          qhi[nt][2 * j + hs][half] = h01 | (h23 << 16);
-          qlo[nt][2 * j + hs][half] = l01 | (l23 << 16);
-        }
-  }
 
-  // ---- per accumulator row (8nt + 2c + e): causal limit and score scale
-  const float kscale = __ldg(p.k_scale + h) * p.qk_scale_log2;
+  // per-portion state (re-initialised for every portion)
+  uint32_t qhi[NT][KSTEP][2], qlo[NT][KSTEP][2];
   int lim[NT][2];
   float scale2[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = row0 + 8 * nt + 2 * c + e;
-      lim[nt][e] = (r < Rtot) ? (L - p.q_len + r / p.G) : (L - 1);
-      const float a = __shfl_sync(kFull, alpha_row[nt], 4 * (2 * c + e));
-      scale2[nt][e] = kscale / a;
-    }
-  const int min_lim = L - p.q_len + row0 / p.G;
-
+  int min_lim = 0;
   float m_run[NT][2], l_run[NT][2];
   float acc[MT][NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-  }
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 
   // this lane's K operand words of one 16-token K tile: rows g8 and g8 + 8,
   // 16-byte chunks 4j + c (D = 128: odd rows fetch their chunks in the other
@@ -439,10 +554,22 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         const uint32_t c1 = hs ? kb[1][j].z : kb[1][j].x, c3 = hs ? kb[1][j].w : kb[1][j].y;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          mma_e4m3(ah[nt], a0, a1, a2, a3, qhi[nt][ks][0], qhi[nt][ks][1]);
-          mma_e4m3(bh[nt], c0, c1, c2, c3, qhi[nt][ks][0], qhi[nt][ks][1]);
-          mma_e4m3(al[nt], a0, a1, a2, a3, qlo[nt][ks][0], qlo[nt][ks][1]);
-          mma_e4m3(bl[nt], c0, c1, c2, c3, qlo[nt][ks][0], qlo[nt][ks][1]);
+          if constexpr (PK) {
+            // packed hi | lo columns; even and odd k-steps go to separate
+            // accumulators so that four chains still interleave
+            if (hs == 0) {
+              mma_e4m3(ah[nt], a0, a1, a2, a3, qhi[nt][ks][0], qhi[nt][ks][1]);
+              mma_e4m3(bh[nt], c0, c1, c2, c3, qhi[nt][ks][0], qhi[nt][ks][1]);
+            } else {
+              mma_e4m3(al[nt], a0, a1, a2, a3, qhi[nt][ks][0], qhi[nt][ks][1]);
+              mma_e4m3(bl[nt], c0, c1, c2, c3, qhi[nt][ks][0], qhi[nt][ks][1]);
+            }
+          } else {
+            mma_e4m3(ah[nt], a0, a1, a2, a3, qhi[nt][ks][0], qhi[nt][ks][1]);
+            mma_e4m3(bh[nt], c0, c1, c2, c3, qhi[nt][ks][0], qhi[nt][ks][1]);
+            mma_e4m3(al[nt], a0, a1, a2, a3, qlo[nt][ks][0], qlo[nt][ks][1]);
+            mma_e4m3(bl[nt], c0, c1, c2, c3, qlo[nt][ks][0], qlo[nt][ks][1]);
+          }
         }
       }
 #pragma unroll
@@ -451,14 +578,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       for (int e = 0; e < 4; ++e) {
         sa[nt][e] = ah[nt][e] + al[nt][e];
         sb[nt][e] = bh[nt][e] + bl[nt][e];
+        if constexpr (PK) {  // column 2c + e holds hi, column 2c + e ^ 4 lo: add them
+          sa[nt][e] += __shfl_xor_sync(kFull, sa[nt][e], 2);
+          sb[nt][e] += __shfl_xor_sync(kFull, sb[nt][e], 2);
+        }
       }
   };
 
-  auto compute_unit = [&](int i, const uint8_t* stage) {
-    const int t0 = unit_t0(i);
-    const int k = 2 * (stream + NSTREAM * i);
-    const int nvA = (piece_of(k) >= 0) ? min(16, t_end - t0) : 0;
-    const int nvB = (piece_of(k + 1) >= 0) ? min(16, t_end - t0 - 16) : 0;
+  auto compute_unit = [&](int t0, int nvA, int nvB, const uint8_t* stage) {
     float sa[NT][4], sb[NT][4];
     qk_unit(stage, sa, sb);
 
@@ -539,6 +666,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       const uint32_t yb = movmatrix_trans(pack_f16x2(pb[2], pb[3]));
       split_e4m3x4(xa, ya, pbhi[nt][0], pblo[nt][0]);
       split_e4m3x4(xb, yb, pbhi[nt][1], pblo[nt][1]);
+      if constexpr (PK) {  // B columns 0-3: hi parts, 4-7: lo parts of the same rows
+        if (g8 >= 4) {
+          pbhi[nt][0] = pblo[nt][0];
+          pbhi[nt][1] = pblo[nt][1];
+        }
+      }
     }
 
     // O^T += V^T . P^T (A7): m-tile mt = head dims 16mt + {g8, g8 + 8}
@@ -560,185 +693,334 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         mma_e4m3(acc[mt][nt], a0, a1, a2, a3, pbhi[nt][0], pbhi[nt][1]);
-        mma_e4m3(acc[mt][nt], a0, a1, a2, a3, pblo[nt][0], pblo[nt][1]);
+        if constexpr (!PK) mma_e4m3(acc[mt][nt], a0, a1, a2, a3, pblo[nt][0], pblo[nt][1]);
       }
     }
   };
 
-  // ---- main loop over this stream's units through the staging ring
-  int consumed = 0;
+  int i_next = 0;  // next stream-local unit to consume
   bool aborted = false;
+  int n_cut = 0, cut0 = 0, cut1 = 0;  // portions whose segment other CTAs share (<= 2)
 #pragma unroll 1
-  for (int i = 0; i < n_my; ++i) {
-    const int st = i % S;
-    const uint32_t par = (uint32_t)((i / S) & 1);
-    if (!mbar_wait_bounded(&full_bar[stream * S + st], par, kWaitLimitNs)) {
-      aborted = true;
-      break;
+  for (int pi = 0; pi < n_port; ++pi) {
+    const Portion P = s_port[pi];
+    const int b = P.b, seg = P.seg, L = P.L;
+    const int h = seg / RB, rg = seg % RB;
+    const int cta_row0 = rg * RC;
+    const int rows_cta = min(RC, Rtot - cta_row0);
+    const int row0 = cta_row0 + rbw * RW;  // this warp's first row
+    const int kb = P.k0, ke = port_end(pi);
+    const bool whole = (P.c_first == P.c_last);
+    if (!whole) {
+      if (n_cut == 0) cut0 = pi; else cut1 = pi;
+      n_cut = min(n_cut + 1, 2);
     }
-    consumed = i + 1;
-    if (row0 < Rtot) compute_unit(i, ring + (size_t)(stream * S + st) * STAGE);
-    __syncwarp();
-    if constexpr (RBG > 1) {
-      if (lane == 0) mbar_arrive(&empty_bar[stream * S + st]);
-    }
-    if (producer && i + S < n_my) {
-      if constexpr (RBG > 1) {
-        if (!mbar_wait_bounded(&empty_bar[stream * S + st], par, kWaitLimitNs)) {
-          aborted = true;
-        }
-      }
-      if (!aborted) {
-        fence_proxy_async_smem();
-        issue(i + S);
-      }
-    }
-    if (__any_sync(kFull, aborted)) break;
-  }
-  if (__any_sync(kFull, aborted)) {
-    if (lane == 0) atomicOr(p.err, ATLAS_DEVERR_TIMEOUT);
-    for (int i = consumed; i < n_my && i < consumed + S; ++i)
-      mbar_wait_bounded(&full_bar[stream * S + i % S], (uint32_t)((i / S) & 1), kWaitLimitNs);
-  }
 
-  // ---- row sums over the token lanes
-  float l_full[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float l = l_run[nt][e];
-      l += __shfl_xor_sync(kFull, l, 4);
-      l += __shfl_xor_sync(kFull, l, 8);
-      l += __shfl_xor_sync(kFull, l, 16);
-      l_full[nt][e] = l;
-    }
-  const float vs = __ldg(p.v_scale + h);
-  const int rows_all = p.q_len * p.Hq;
+    // groups in flight: portions pi and (if it exists) pi + 1; wait for pi's
+    if (pi + 1 < n_port) cp_async_wait_group1(); else cp_async_wait_all();
+    __syncthreads();  // this portion's Q rows are in buffer pi % kQBuf
+    if (pi + 2 < n_port) prefetch_q(pi + 2);  // into the buffer portion pi - 1 used
+    const __nv_bfloat16* qb = s_q + (size_t)(pi % kQBuf) * rows_max * D;
 
-  if constexpr (NSTREAM == 1) {
-    // one stream: every warp owns its rows outright; store from registers
-    if (row0 < Rtot) {
+    // ---- Q^T fragments as E4M3 hi + lo with a per-row power-of-two scale
+    // B operand of k-step s = 2j + hs: b0 = dims 64j+16c+8hs+{0..3}, b1 = +{4..7}.
+    float alpha_row[NT];  // the scale of row 8nt + g8
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
+      // row within the row group (PK: lanes g8 and g8 + 4 both prepare row g8 % 4)
+      const int lr = PK ? (g8 & 3) : rbw * RW + 8 * nt + g8;
+      float x[NCH][16];
+      if (cta_row0 + lr < Rtot) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int r = row0 + 8 * nt + 2 * c + e;
-          if (r >= Rtot) continue;
-          const int i = r / p.G, hq = h * p.G + r % p.G;
-          const int grow = i * p.Hq + hq;
-          const float den = l_full[nt][e];
-          const float inv = den > 0.f ? 1.f / den : 0.f;
-          if (n_split_b == 1) {
-            __nv_bfloat16* orow = p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * D;
+        for (int j = 0; j < NCH; ++j) {
+          const uint4* src = reinterpret_cast<const uint4*>(qb + lr * D + j * 64 + 16 * c);
+          const uint4 w0 = src[0], w1 = src[1];
+          const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              orow[16 * mt + g8] = __float2bfloat16_rn(acc[mt][nt][e] * inv * vs);
-              orow[16 * mt + g8 + 8] = __float2bfloat16_rn(acc[mt][nt][e + 2] * inv * vs);
-            }
-          } else {
-            const size_t base = ((size_t)b * p.num_splits + split) * rows_all + grow;
-            float* prow = p.part_o + base * D;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              prow[16 * mt + g8] = acc[mt][nt][e] * inv;
-              prow[16 * mt + g8 + 8] = acc[mt][nt][e + 2] * inv;
-            }
-            if (g8 == 0) p.part_lse[base] = den > 0.f ? m_run[nt][e] + __log2f(den) : -INFINITY;
+          for (int k = 0; k < 8; ++k) {
+            x[j][2 * k] = __uint_as_float(wv[k] << 16);
+            x[j][2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
           }
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < NCH; ++j)
+#pragma unroll
+          for (int k = 0; k < 16; ++k) x[j][k] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[j][k]));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      // a = 2^(135 - e) puts amax in [256, 512); halve it if amax * a > 448
+      const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+      float a = 1.f;
+      if (amax > 0.f) {
+        const int ex = min(254, max(1, 262 - e));
+        a = __uint_as_float((uint32_t)ex << 23);
+        if (amax * a > 448.f) a *= 0.5f;
+      }
+      alpha_row[nt] = a;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j)
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs)
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int k0 = 8 * hs + 4 * half;
+            const float y0 = x[j][k0] * a, y1 = x[j][k0 + 1] * a;
+            const float y2 = x[j][k0 + 2] * a, y3 = x[j][k0 + 3] * a;
+            const uint32_t h01 = f32x2_to_e4m3x2(y0, y1), h23 = f32x2_to_e4m3x2(y2, y3);
+            const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
+            const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
+            const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
+            const uint32_t l01 = f32x2_to_e4m3x2(y0 - b01.x, y1 - b01.y);
+            const uint32_t l23 = f32x2_to_e4m3x2(y2 - b23.x, y3 - b23.y);
+            // PK: lanes g8 < 4 feed the hi columns, lanes g8 >= 4 the lo columns
+            qhi[nt][2 * j + hs][half] = (PK && g8 >= 4) ? (l01 | (l23 << 16)) : (h01 | (h23 << 16));
+            qlo[nt][2 * j + hs][half] = l01 | (l23 << 16);
+          }
     }
-  } else {
-    __syncthreads();  // every warp is done with the ring: reuse it for the combine
-    float* s_m = reinterpret_cast<float*>(ring);
-    float* s_l = s_m + NSTREAM * RC;
-    float* s_o = s_l + NSTREAM * RC;
+    // per accumulator row (8nt + 2c + e): causal limit and score scale
+    const float kscale = P.k_scale * p.qk_scale_log2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int lr = rbw * RW + 8 * nt + 2 * c + e;
-        if (g8 == 0) {
-          s_m[stream * RC + lr] = m_run[nt][e];
-          s_l[stream * RC + lr] = l_full[nt][e];
-        }
+        // the row of accumulator column 2c + e (PK: columns c and c ^ 2 are one row)
+        const int rl = PK ? 2 * (c & 1) + e : 8 * nt + 2 * c + e;
+        const int r = row0 + rl;
+        lim[nt][e] = (r < Rtot) ? (L - p.q_len + r / p.G) : (L - 1);
+        const float a = __shfl_sync(kFull, alpha_row[nt], 4 * (rl - 8 * nt));
+        scale2[nt][e] = kscale / a;
       }
+    min_lim = L - p.q_len + row0 / p.G;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.f;
+    }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int lr = rbw * RW + 8 * nt + 2 * c + (e & 1);
-          const int d = 16 * mt + g8 + ((e & 2) ? 8 : 0);
-          s_o[((size_t)stream * RC + lr) * D + d] = acc[mt][nt][e];
-        }
-    __syncthreads();
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
 
-    // combine the streams; write output (one split) or the split partial
-    for (int idx = tid; idx < rows_cta * D; idx += kThreads) {
-      const int lr = idx / D, d = idx % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NSTREAM; ++w) M = fmaxf(M, s_m[w * RC + lr]);
-      float den = 0.f, num = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < NSTREAM; ++w) {
-          const float f = fast_exp2(s_m[w * RC + lr] - M);
-          den += f * s_l[w * RC + lr];
-          num += f * s_o[((size_t)w * RC + lr) * D + d];
-        }
+    // ---- this stream's units of the portion: k in [kb, ke), k = stream + NSTREAM*i
+#pragma unroll 1
+    for (; !aborted; ++i_next) {
+      const int k = stream + NSTREAM * i_next;
+      if (k >= ke) break;
+      const int st = i_next % S;
+      const uint32_t par = (uint32_t)((i_next / S) & 1);
+      if (!mbar_wait_bounded(&full_bar[stream * S + st], par, kWaitLimitNs)) {
+        aborted = true;
+        break;
       }
-      const int r = cta_row0 + lr;
-      const int i = r / p.G, hq = h * p.G + r % p.G;
-      const int grow = i * p.Hq + hq;
-      if (n_split_b == 1) {
-        p.out[(((size_t)b * p.q_len + i) * p.Hq + hq) * D + d] =
-            __float2bfloat16_rn(den > 0.f ? num / den * vs : 0.f);
-      } else {
-        const size_t base = ((size_t)b * p.num_splits + split) * rows_all + grow;
-        p.part_o[base * D + d] = (den > 0.f) ? num / den : 0.f;
-        // the log2-sum-exp carries the 2^8 factor of p; it cancels in the merge
-        if (d == 0) p.part_lse[base] = (den > 0.f) ? M + __log2f(den) : -INFINITY;
+      if (row0 < Rtot) {
+        const int2 pc = s_pieces[k];
+        const int t0 = kUnit * (P.ua + k - kb);
+        const int nvA = pc.x >= 0 ? min(16, L - t0) : 0;
+        const int nvB = pc.y >= 0 ? min(16, L - t0 - 16) : 0;
+        compute_unit(t0, nvA, nvB, ring + (size_t)(stream * S + st) * STAGE);
+      }
+      __syncwarp();
+      if constexpr (RBG > 1) {
+        if (lane == 0) mbar_arrive(&empty_bar[stream * S + st]);
+      }
+      if (producer && i_next + S < n_my) {
+        if constexpr (RBG > 1) {
+          if (!mbar_wait_bounded(&empty_bar[stream * S + st], par, kWaitLimitNs)) aborted = true;
+        }
+        // the stage's readers are done: RBG = 1, their loads fed this warp's MMAs
+        // before the __syncwarp; RBG > 1, the empty barrier ordered them
+        if (!aborted) issue(i_next + S);
+      }
+      if (__any_sync(kFull, aborted)) aborted = true;
+    }
+
+    // ---- PK: O's hi and lo columns (lanes c and c ^ 2) add up to the row's O
+    if constexpr (PK) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][0][e] += __shfl_xor_sync(kFull, acc[mt][0][e], 2);
+    }
+    // ---- row sums over the token lanes
+    float l_full[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = l_run[nt][e];
+        l += __shfl_xor_sync(kFull, l, 4);
+        l += __shfl_xor_sync(kFull, l, 8);
+        l += __shfl_xor_sync(kFull, l, 16);
+        l_full[nt][e] = l;
+      }
+
+    // ---- where the portion's result goes: the output, or partial slot
+    // (segment + CTA) when other CTAs hold parts of the segment
+    const int seg_idx = b * Hs + seg;
+    const float vs = P.v_scale;
+    const size_t slot = (size_t)seg_idx + cid;
+
+    if constexpr (NSTREAM == 1) {
+      // one stream: every warp owns its rows outright; store from registers
+      if (row0 < Rtot) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int lr = rbw * RW + 8 * nt + 2 * c + e;
+            const int r = cta_row0 + lr;
+            if (r >= Rtot) continue;
+            const int i = r / p.G, hq = h * p.G + r % p.G;
+            const float den = l_full[nt][e];
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            if (whole) {
+              __nv_bfloat16* orow = p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * D;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                orow[16 * mt + g8] = __float2bfloat16_rn(acc[mt][nt][e] * inv * vs);
+                orow[16 * mt + g8 + 8] = __float2bfloat16_rn(acc[mt][nt][e + 2] * inv * vs);
+              }
+            } else {
+              float* prow = p.part_o + (slot * RC + lr) * D;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                prow[16 * mt + g8] = acc[mt][nt][e] * inv;
+                prow[16 * mt + g8 + 8] = acc[mt][nt][e + 2] * inv;
+              }
+              if (g8 == 0)
+                p.part_lse[slot * RC + lr] = den > 0.f ? m_run[nt][e] + __log2f(den) : -INFINITY;
+            }
+          }
+      }
+    } else {
+      // streams leave (m, l, O / l) of their rows in shared memory; all
+      // threads combine them (O / l is at most max|v| <= 448: half is enough)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int lr = PK ? 2 * c + e : rbw * RW + 8 * nt + 2 * c + e;
+          if (lr < rows_cta && (!PK || c < 2)) {
+            const float den = l_full[nt][e];
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            if (g8 == 0) {
+              s_cm[stream * rows_max + lr] = m_run[nt][e];
+              s_cl[stream * rows_max + lr] = den;
+            }
+            __half* orow = s_co + ((size_t)stream * rows_max + lr) * D;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              orow[16 * mt + g8] = __float2half_rn(acc[mt][nt][e] * inv);
+              orow[16 * mt + g8 + 8] = __float2half_rn(acc[mt][nt][e + 2] * inv);
+            }
+          }
+        }
+      __syncthreads();
+      for (int idx = tid; idx < rows_cta * D; idx += kThreads) {
+        const int lr = idx / D, d = idx - lr * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NSTREAM; ++w) M = fmaxf(M, s_cm[w * rows_max + lr]);
+        float den = 0.f, num = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < NSTREAM; ++w) {
+            const float f = fast_exp2(s_cm[w * rows_max + lr] - M) * s_cl[w * rows_max + lr];
+            den += f;
+            num += f * __half2float(s_co[((size_t)w * rows_max + lr) * D + d]);
+          }
+        }
+        const int r = cta_row0 + lr;
+        const int i = r / p.G, hq = h * p.G + r % p.G;
+        if (whole) {
+          p.out[(((size_t)b * p.q_len + i) * p.Hq + hq) * D + d] =
+              __float2bfloat16_rn(den > 0.f ? num / den * vs : 0.f);
+        } else {
+          p.part_o[(slot * RC + lr) * D + d] = (den > 0.f) ? num / den : 0.f;
+          // the log2-sum-exp carries the 2^8 factor of p; it cancels in the merge
+          if (d == 0) p.part_lse[slot * RC + lr] = (den > 0.f) ? M + __log2f(den) : -INFINITY;
+        }
       }
     }
+    // the combine buffer is free for the next portion; a timeout anywhere stops the CTA
+    if (__syncthreads_or(aborted)) {
+      aborted = true;
+      break;
+    }
   }
-  if (n_split_b == 1) return;
 
-  // ---- last CTA of this (b, h, row group) merges the splits (A8 -> A9)
-  __threadfence();
-  __syncthreads();
-  int32_t* counter = p.counters + ((size_t)b * p.Hkv + h) * p.row_blocks + grp;
-  if (tid == 0) s_is_last = (atomicAdd(counter, 1) == n_split_b - 1);
-  __syncthreads();
-  if (!s_is_last) return;
-  __threadfence();
+  if (aborted) {
+    if (lane == 0) atomicOr(p.err, ATLAS_DEVERR_TIMEOUT);
+    // drain this stream's loads still in flight (issued: i < min(n_my, i_next + S))
+    for (int i = i_next; i < n_my && i < i_next + S; ++i)
+      mbar_wait_bounded(&full_bar[stream * S + i % S], (uint32_t)((i / S) & 1), kWaitLimitNs);
+    cp_async_wait_all();
+    return;
+  }
+  if (n_cut == 0) return;
 
-  for (int lr = warp; lr < rows_cta; lr += kWarps) {
-    const int r = cta_row0 + lr;
-    const int i = r / p.G, hq = h * p.G + r % p.G;
-    const int grow = i * p.Hq + hq;
-    const float* lse = p.part_lse + (size_t)b * p.num_splits * rows_all + grow;
-    float M = -INFINITY;
-    for (int sp = lane; sp < n_split_b; sp += 32) M = fmaxf(M, __ldcg(lse + (size_t)sp * rows_all));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    float den = 0.f;
-    for (int sp = lane; sp < n_split_b; sp += 32)
-      den += fast_exp2(__ldcg(lse + (size_t)sp * rows_all) - M);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(kFull, den, o);
-    const float inv = vs / den;
-    for (int d0 = lane * 4; d0 < D; d0 += 128) {
-      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < n_split_b; ++sp) {
-        const float wgt = fast_exp2(__ldcg(lse + (size_t)sp * rows_all) - M);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(
-            p.part_o + (((size_t)b * p.num_splits + sp) * rows_all + grow) * D + d0));
-        o4.x += wgt * v.x; o4.y += wgt * v.y; o4.z += wgt * v.z; o4.w += wgt * v.w;
+  // ---- segments shared with other CTAs (A8 -> A9): one completion counter per
+  // segment; the CTA that finishes a segment last merges its partial slots.
+  // Done once at the end, so that no portion waits on a fence or an atomic.
+  __threadfence();
+  for (int q = 0; q < n_cut; ++q) {
+    const Portion P = s_port[q == 0 ? cut0 : cut1];
+    const int seg_idx = P.b * Hs + P.seg;
+    const int h = P.seg / RB, cta_row0 = (P.seg % RB) * RC;
+    const int rows_cta = min(RC, Rtot - cta_row0);
+    int32_t* counter = p.counters + seg_idx;
+    __syncthreads();  // every thread's partial stores are fenced; s_is_last is free
+    if (tid == 0) s_is_last = (atomicAdd(counter, 1) == P.c_last - P.c_first);
+    __syncthreads();
+    if (!s_is_last) continue;
+    __threadfence();
+    const size_t s0 = (size_t)seg_idx + P.c_first;
+    const int n_slots = P.c_last - P.c_first + 1;
+    // per row: reference M and denominator over the slots' log2-sum-exp values
+    for (int lr = tid; lr < rows_cta; lr += kThreads) {
+      float M = -INFINITY, den = 0.f;
+      for (int sl = 0; sl < n_slots; ++sl) {
+        const float v = __ldcg(p.part_lse + (s0 + sl) * RC + lr);
+        if (v == -INFINITY) continue;
+        if (v > M) {
+          den = den * fast_exp2(M - v) + 1.f;
+          M = v;
+        } else {
+          den += fast_exp2(v - M);
+        }
       }
-      __nv_bfloat16* dst = p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * D + d0;
+      s_rowM[lr] = M;
+      s_rowD[lr] = den;
+    }
+    __syncthreads();
+    const float vs = P.v_scale;
+    constexpr int C4 = D / 4;
+    for (int idx = tid; idx < rows_cta * C4; idx += kThreads) {
+      const int lr = idx / C4, d0 = 4 * (idx - lr * C4);
+      const float M = s_rowM[lr], den = s_rowD[lr];
+      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (den > 0.f) {
+#pragma unroll 4
+        for (int sl = 0; sl < n_slots; ++sl) {
+          const float wgt = fast_exp2(__ldcg(p.part_lse + (s0 + sl) * RC + lr) - M);
+          const float4 v =
+              __ldcg(reinterpret_cast<const float4*>(p.part_o + ((s0 + sl) * RC + lr) * D + d0));
+          o4.x += wgt * v.x; o4.y += wgt * v.y; o4.z += wgt * v.z; o4.w += wgt * v.w;
+        }
+      }
+      const float inv = den > 0.f ? vs / den : 0.f;
+      const int r = cta_row0 + lr;
+      const int i = r / p.G, hq = h * p.G + r % p.G;
+      __nv_bfloat16* dst = p.out + (((size_t)P.b * p.q_len + i) * p.Hq + hq) * D + d0;
       const __nv_bfloat162 lo = __floats2bfloat162_rn(o4.x * inv, o4.y * inv);
       const __nv_bfloat162 hi = __floats2bfloat162_rn(o4.z * inv, o4.w * inv);
       uint2 pk;
@@ -746,45 +1028,87 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       pk.y = *reinterpret_cast<const uint32_t*>(&hi);
       *reinterpret_cast<uint2*>(dst) = pk;
     }
+    if (tid == 0) *counter = 0;  // ready for the next call on this stream
   }
-  if (tid == 0) *counter = 0;  // ready for the next call on this stream
 }
 
-template <int D, int NT, int RBG, int S>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t stream) {
-  const size_t smem = Smem<D, S, kWarps / RBG, 8 * NT * RBG>::total(p.split_tokens);
-  auto kern = paged_decode_fp8_kernel<D, NT, RBG, S>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.num_splits * p.row_blocks, p.Hkv, p.B);
-  kern<<<grid, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
-}
+// ------------------------------------------------------------------- launching
 
-template <int D, int NT, int RBG>
-cudaError_t launch_s(const DecodeParams& p, int stages, cudaStream_t stream) {
-  if (stages == 2) return launch_t<D, NT, RBG, 2>(p, stream);
-  if (stages == 3) return launch_t<D, NT, RBG, 3>(p, stream);
+template <int D, int NT, int RBG, int S, bool PK>
+struct Cfg {
+  static constexpr auto kernel() { return paged_decode_fp8_kernel<D, NT, RBG, S, PK>; }
+};
+
+// Calls f(Cfg<...>{}) for the instantiation that serves these parameters.
+template <int D, int NT, int RBG, bool PK, class F>
+cudaError_t with_stages(int stages, F&& f) {
+  if (stages == 2) return f(Cfg<D, NT, RBG, 2, PK>{});
+  if (stages == 3) return f(Cfg<D, NT, RBG, 3, PK>{});
   return cudaErrorInvalidValue;
 }
-
-template <int D>
-cudaError_t launch_d(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
-                     cudaStream_t stream) {
-  if (rows_per_warp == 8 && rbg == 1) return launch_s<D, 1, 1>(p, stages, stream);
-  if (rows_per_warp == 16 && rbg == 1) return launch_s<D, 2, 1>(p, stages, stream);
-  if (rows_per_warp == 16 && rbg == 2) return launch_s<D, 2, 2>(p, stages, stream);
-  if (rows_per_warp == 16 && rbg == 4) return launch_s<D, 2, 4>(p, stages, stream);
+template <int D, class F>
+cudaError_t with_rows(int rows_per_warp, int rbg, int stages, F&& f) {
+  if (rows_per_warp == 4 && rbg == 1) return with_stages<D, 1, 1, true>(stages, f);
+  if (rows_per_warp == 8 && rbg == 1) return with_stages<D, 1, 1, false>(stages, f);
+  if (rows_per_warp == 16 && rbg == 1) return with_stages<D, 2, 1, false>(stages, f);
+  if (rows_per_warp == 16 && rbg == 2) return with_stages<D, 2, 2, false>(stages, f);
+  if (rows_per_warp == 16 && rbg == 4) return with_stages<D, 2, 4, false>(stages, f);
+  return cudaErrorInvalidValue;
+}
+template <class F>
+cudaError_t with_kernel(int D, int rows_per_warp, int rbg, int stages, F&& f) {
+  if (D == 128) return with_rows<128>(rows_per_warp, rbg, stages, f);
+  if (D == 64) return with_rows<64>(rows_per_warp, rbg, stages, f);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units,
+                             int max_portions) {
+  return smem_plan(D, stages, kWarps / rbg, rows, max_units, max_portions).total;
+}
+
+void decode_fp8_fit_grid(int D, int rows, int sms, DecodeLaunch& L) {
+  if (L.per_segment) return;
+  for (int it = 0; it < 4; ++it) {
+    const size_t smem = decode_fp8_smem_bytes(D, L.stages, L.rbg, rows, L.max_units,
+                                              L.max_portions);
+    int occ = 0;
+    const cudaError_t e = with_kernel(D, L.rows_per_warp, L.rbg, L.stages, [&](auto cfg) {
+      auto kern = decltype(cfg)::kernel();
+      cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (r != cudaSuccess) return r;
+      return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+    });
+    if (e != cudaSuccess || occ <= 0) {
+      cudaGetLastError();
+      return;  // the launch reports the problem
+    }
+    const long long resident = (long long)sms * occ * L.waves;
+    if (L.grid <= resident) return;
+    const long long mu = (L.units_max + resident - 1) / resident;
+    if (mu > kMaxUnitsPerCta) return;
+    L.grid = resident;
+    L.max_units = (int)mu;
+    L.max_portions = (int)(L.segs < mu ? L.segs : mu);
+  }
+}
+
 cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
-                              cudaStream_t stream) {
-  if (p.D == 128) return launch_d<128>(p, rows_per_warp, rbg, stages, stream);
-  if (p.D == 64) return launch_d<64>(p, rows_per_warp, rbg, stages, stream);
-  return cudaErrorInvalidValue;
+                              long long grid, cudaStream_t stream) {
+  if (grid < 1 || grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  const int rows = min(rows_per_warp * rbg, p.q_len * p.G);
+  const size_t smem = decode_fp8_smem_bytes(p.D, stages, rbg, rows, p.max_units, p.max_portions);
+  return with_kernel(p.D, rows_per_warp, rbg, stages, [&](auto cfg) {
+    auto kern = decltype(cfg)::kernel();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  });
 }
 
 }  // namespace atlas

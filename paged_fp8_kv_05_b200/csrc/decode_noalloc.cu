@@ -15,10 +15,10 @@
 // contents; each call clears the counters and the error word (the only parts
 // that must start at zero) with cudaMemsetAsync on its stream before the
 // launch.  Calls whose kernels overlap on the GPU (different streams, no
-// ordering) race on the array.  If the split-KV partials of a call would not
-// fit, the call uses longer splits (down to one split per sequence); a call
-// whose counters alone would not fit, or that would need splits longer than
-// 65536 tokens, is rejected with ATLAS_ERR_WORKSPACE.
+// ordering) race on the array.  If the split-KV partials of the balanced
+// partition would not fit, the call runs one CTA per (sequence, KV head, row
+// group) segment, which writes no partials; a call that would then need a
+// segment longer than 65536 tokens is rejected with ATLAS_ERR_WORKSPACE.
 // The first call on a device looks up the array's device address
 // (cudaGetSymbolAddress) with that device current; make that first call
 // before any stream capture.  Device-side checks still zero the rows of an
@@ -77,29 +77,7 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
     return ATLAS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_pages) || !aligned16(v_pages))
     return ATLAS_ERR_INVALID_ARG;
-  if (batch > 65535 || num_kv_heads > 65535) return ATLAS_ERR_UNSUPPORTED;
 
-  // launch shape: the same choice of rows per warp / warps per K/V stream as
-  // the pool-based entry point
-  const int G = num_q_heads / num_kv_heads;
-  const int R = q_len * G;
-  const int rows_per_warp = (R <= 8) ? 8 : 16;
-  const int rbg = (R <= 16) ? 1 : (R <= 32 ? 2 : 4);
-  const int rows_per_cta = rows_per_warp * rbg;
-  const int row_blocks = (R + rows_per_cta - 1) / rows_per_cta;
-  const int stages = (rbg == 1) ? 2 : 3;
-  const int rows_all = q_len * num_q_heads;
-
-  // scratch layout: [error word][counters][log2-sum-exp][O partials]
-  const size_t counters_bytes =
-      align_up((size_t)batch * num_kv_heads * row_blocks * sizeof(int32_t), kAlign);
-  if (kAlign + counters_bytes > kScratchBytes) return ATLAS_ERR_WORKSPACE;
-  const size_t room = kScratchBytes - kAlign - counters_bytes;
-  const size_t per_split = (size_t)batch * rows_all * (head_dim + 1) * sizeof(float) + 2 * kAlign;
-
-  // split size: about two waves of 4 resident CTAs per SM if every sequence
-  // were max_seq_len long, 256..8192 tokens, then lengthened until the
-  // partials fit in the scratch
   int sms = 148;
   {
     int dev = 0, n = 0;
@@ -107,32 +85,32 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
       sms = n;
   }
-  const long long units = (long long)batch * num_kv_heads * row_blocks;
-  long long want = ((long long)sms * 8 + units - 1) / units;
-  if (want < 1) want = 1;
-  long long T = (max_seq_len + want - 1) / want;
-  T = (T + 63) / 64 * 64;
-  if (T < 256) T = 256;
-  if (T > 8192) T = 8192;
-  int num_splits = (int)((max_seq_len + T - 1) / T);
-  if (num_splits > 1 && (size_t)num_splits * per_split > room) {
-    const long long fit = (long long)(room / per_split);
-    if (fit <= 1) {
-      num_splits = 1;
-      T = ((long long)max_seq_len + 63) / 64 * 64;
-    } else {
-      T = ((max_seq_len + fit - 1) / fit + 63) / 64 * 64;
-      num_splits = (int)((max_seq_len + T - 1) / T);
-    }
+  const int R = q_len * (num_q_heads / num_kv_heads);
+
+  // the balanced partition of the pool-based entry point if its scratch --
+  // [error word][counters][log2-sum-exp][O partials] -- fits; else one CTA per
+  // segment, which needs only the error word
+  atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len,
+                                             max_seq_len, sms, 0, 0, false);
+  atlas::decode_fp8_fit_grid(head_dim, R < L.rows_per_cta ? R : L.rows_per_cta, sms, L);
+  size_t counters_off = kAlign;
+  size_t lse_off = counters_off + align_up((size_t)L.segs * sizeof(int32_t), kAlign);
+  const size_t rows = (size_t)L.slots * L.rows_per_cta;
+  size_t o_off = lse_off + align_up(rows * sizeof(float), kAlign);
+  size_t clear = lse_off;  // error word + counters
+  if (o_off + rows * head_dim * sizeof(float) > kScratchBytes) {
+    L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len, max_seq_len, sms, 0, 0, true);
+    // one segment's unit table lives in shared memory: bound its length
+    if (L.max_units > 2 * atlas::kMaxUnitsPerCta) return ATLAS_ERR_WORKSPACE;
+    lse_off = o_off = counters_off;
+    clear = kAlign;
   }
-  if (num_splits == 1 && T < max_seq_len) T = ((long long)max_seq_len + 63) / 64 * 64;
-  // one split holds its page-piece table in shared memory: bound its length
-  if (T > 65536) return ATLAS_ERR_WORKSPACE;
+  if (L.grid > 0x7FFFFFFFLL) return ATLAS_ERR_UNSUPPORTED;
 
   uint8_t* scratch = static_cast<uint8_t*>(scratch_on_current_device());
   if (!scratch) return ATLAS_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, kAlign + counters_bytes, s) != cudaSuccess) return ATLAS_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, clear, s) != cudaSuccess) return ATLAS_ERR_CUDA;
 
   atlas::DecodeParams p{};  // value-initialised: no fused append unless set
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -144,26 +122,27 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   p.seq_lens = seq_lens;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = reinterpret_cast<int32_t*>(scratch);
-  p.counters = reinterpret_cast<int32_t*>(scratch + kAlign);
-  const size_t lse_bytes = align_up((size_t)batch * num_splits * rows_all * sizeof(float), kAlign);
-  p.part_lse = reinterpret_cast<float*>(scratch + kAlign + counters_bytes);
-  p.part_o = reinterpret_cast<float*>(scratch + kAlign + counters_bytes + lse_bytes);
+  p.counters = reinterpret_cast<int32_t*>(scratch + counters_off);
+  p.part_lse = reinterpret_cast<float*>(scratch + lse_off);
+  p.part_o = reinterpret_cast<float*>(scratch + o_off);
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
-  p.G = G;
+  p.G = num_q_heads / num_kv_heads;
   p.q_len = q_len;
   p.D = head_dim;
   p.ps = page_size;
   p.num_pages = num_pages;
   p.max_blocks = max_blocks_per_seq;
-  p.split_tokens = (int)T;
-  p.num_splits = num_splits;
-  p.row_blocks = row_blocks;
+  p.max_seq_len = max_seq_len;
+  p.row_blocks = L.row_blocks;
+  p.max_units = L.max_units;
+  p.max_portions = L.max_portions;
+  p.per_segment = L.per_segment;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
   p.k_new = nullptr;  // decode only
   p.v_new = nullptr;
-  cudaError_t e = atlas::launch_decode_fp8(p, rows_per_warp, rbg, stages, s);
+  cudaError_t e = atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid, s);
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

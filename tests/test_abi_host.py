@@ -50,13 +50,18 @@ def test_status_strings_and_version():
 
 
 def test_workspace_bytes():
-    n = ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 256)
-    # header + counters + lse + O for 16 splits
-    assert n >= 256 + 32 * 32 * 4 + 32 * 16 * 32 * (128 + 1) * 4
-    assert ak.atlas_kv_workspace_bytes(32, 1, 32, 96, 4096) == 0        # head_dim
-    assert ak.atlas_kv_workspace_bytes(32, 0, 32, 128, 4096) == 0       # q_len
-    assert (ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 64)
-            > ak.atlas_kv_workspace_bytes(32, 1, 32, 128, 4096, 256))
+    # batch 32, 8 KV heads, group 4 -> 256 segments of 4 rows; 4096 tokens = 128
+    # units each; 256-token ranges -> 32768 / 8 = 4096 CTAs; one partial slot per
+    # segment plus one per CTA, each 4 rows x (128 + 1) floats
+    n = ak.atlas_kv_workspace_bytes(32, 1, 32, 8, 128, 4096, 256)
+    segs, ctas = 32 * 8, 32 * 8 * 128 // 8
+    assert n >= 256 + segs * 4 + (segs + ctas) * 4 * (128 + 1) * 4
+    assert ak.atlas_kv_workspace_bytes(32, 1, 32, 8, 96, 4096) == 0     # head_dim
+    assert ak.atlas_kv_workspace_bytes(32, 0, 32, 8, 128, 4096) == 0    # q_len
+    assert ak.atlas_kv_workspace_bytes(32, 1, 32, 6, 128, 4096) == 0    # 32 % 6 != 0
+    assert (ak.atlas_kv_workspace_bytes(32, 1, 32, 8, 128, 4096, 64)
+            > ak.atlas_kv_workspace_bytes(32, 1, 32, 8, 128, 4096, 256)
+            > ak.atlas_kv_workspace_bytes(32, 1, 32, 8, 128, 4096, 0))
 
 
 class _Fake:
@@ -108,13 +113,16 @@ def test_pool_create_ok_and_plan_is_host_only():
         buf = (ctypes.c_int32 * 7)()
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 100, buf, 7) == ak.ATLAS_OK
         plan = dict(zip(ak.PLAN_FIELDS, buf))
-        assert plan["split_tokens"] % 64 == 0 and plan["num_splits"] >= 1
-        assert plan["rows_per_cta"] == 8 and plan["row_blocks"] == 1 and plan["launches"] == 1
+        # 2 x 2 segments of 4 units (100 tokens): 16 units, one per CTA
+        assert plan["split_tokens"] == 32 and plan["num_splits"] == 4
+        assert plan["grid_ctas"] == 16
+        assert plan["rows_per_cta"] == 4 and plan["row_blocks"] == 1 and plan["launches"] == 1
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 5, 100, buf, 7) == ak.ATLAS_OK
         assert buf[3] == 32 and buf[4] == 1           # 5 x 4 rows: two warps of 16 share K/V
         assert ak._lib.atlas_kv_pool_set_split_tokens(h, 128) == ak.ATLAS_OK
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 1000, buf, 7) == ak.ATLAS_OK
-        assert buf[0] == 128 and buf[1] == 8
+        # 4 segments x 32 units in ranges of 4 units: 32 CTAs; a segment meets <= 9
+        assert buf[0] == 128 and buf[1] == 9 and buf[6] == 32
         for bad in (-64, 32, 100, 16384):
             assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
         for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 2, 0), (ak.OPT_STAGES, 0, 0),
