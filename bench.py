@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--split-tokens", type=int, default=0, help="override the split size")
     ap.add_argument("--stages", type=int, default=0, help="override the K/V staging depth")
     ap.add_argument("--waves", type=int, default=0, help="CTAs per resident CTA slot")
+    ap.add_argument("--partition", type=int, default=0, help="0 auto, 1 grid, 2 balanced")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -325,6 +326,8 @@ def ours(args):
         dw.pool.set_option(ak.OPT_STAGES, args.stages)
     if args.waves:
         dw.pool.set_option(ak.OPT_WAVES, args.waves)
+    if args.partition:
+        dw.pool.set_option(ak.OPT_PARTITION, args.partition)
     plan = dw.plan()
     b_dec, b_app = algorithmic_bytes(w)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)

@@ -88,9 +88,11 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
 #define ATLAS_DEVERR_TIMEOUT   0x8   /* decode: a bounded wait for staged K/V ran out      */
 
 /* Fields of atlas_paged_gqa_decode_plan's output array. */
-#define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per CTA range (most any CTA gets)    */
-#define ATLAS_PLAN_NUM_SPLITS    1   /* most CTA ranges one max-length segment spans  */
-#define ATLAS_PLAN_KERNEL        2   /* 1 = FP8 mma.sync kernel (E4M3 tensor cores)    */
+#define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split / per CTA range           */
+#define ATLAS_PLAN_NUM_SPLITS    1   /* splits (grid) or most ranges (balanced) of a  */
+                                     /* max-length segment                            */
+#define ATLAS_PLAN_KERNEL        2   /* FP8 mma.sync kernel (E4M3 tensor cores) with  */
+                                     /* 1 = grid partition, 2 = balanced partition    */
 #define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) per segment        */
 #define ATLAS_PLAN_ROW_BLOCKS    4   /* segments per (sequence, KV head)              */
 #define ATLAS_PLAN_LAUNCHES      5   /* kernel launches per decode call               */
@@ -138,12 +140,12 @@ ATLAS_API atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** pool, int32_t nu
 ATLAS_API atlas_status_t atlas_kv_pool_destroy(atlas_kv_pool_t* pool);
 
 /*
- * Override the partition of later decode calls: CTA ranges of about
- * split_tokens KV tokens (ceil(units / (split_tokens / 32)) CTAs, where units
+ * Override the split length of later decode calls: splits of split_tokens KV
+ * tokens (grid partition), or CTA ranges of about split_tokens tokens
+ * (balanced partition: ceil(units / (split_tokens / 32)) CTAs, where units
  * counts 32-token units as if every sequence were max_seq_len long); 0
- * restores the automatic choice (one range per resident CTA).  Must be 0 or a
- * multiple of 64 in [64, 8192].  Meant for tuning and for split-invariance
- * tests.
+ * restores the automatic choice.  Must be 0 or a multiple of 64 in [64, 8192].
+ * Meant for tuning and for split-invariance tests.
  */
 ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, int32_t split_tokens);
 
@@ -154,6 +156,11 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
                                      /* up to 8 (smaller ranges the hardware schedules    */
                                      /* as slots free up); the workspace must hold the    */
                                      /* extra partial slots (ATLAS_ERR_WORKSPACE if not)  */
+#define ATLAS_OPT_PARTITION      4   /* 0 = auto, 1 = grid (CTA = one split of one      */
+                                     /* (sequence, KV head, row block); the hardware     */
+                                     /* schedules them), 2 = balanced (equal ranges of   */
+                                     /* 32-token units per CTA); auto takes balanced     */
+                                     /* only when one K/V stream serves a whole CTA      */
 
 /*
  * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of
@@ -193,11 +200,12 @@ ATLAS_API atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const 
  * seq_len > max_seq_len gets zero output rows and flags ATLAS_DEVERR_SEQ_LEN; a page id outside
  * [0, num_pages) is skipped (its tokens do not take part) and flags
  * ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
- * Partition: the 32-token units of all (sequence, KV head, row block)
- * segments are cut into equal contiguous ranges, one per CTA, so every CTA
- * streams the same number of KV bytes whatever the length mix; a segment cut
- * by a range boundary is merged by log-sum-exp by the CTA that finishes it
- * last.  A wait that runs out (200 ms) flags ATLAS_DEVERR_TIMEOUT.
+ * Partition (ATLAS_OPT_PARTITION): each (sequence, KV head, row block)
+ * segment is cut into splits of a fixed number of tokens, one CTA each, that
+ * the hardware hands to SMs as they free up; or the 32-token units of all
+ * segments are cut into equal ranges, one per CTA, whatever the length mix.
+ * A segment cut in several parts is merged by log-sum-exp by the CTA that
+ * finishes it last.  A wait that runs out (200 ms) flags ATLAS_DEVERR_TIMEOUT.
  */
 ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q,
                                       const void* k_pages, const void* v_pages,
@@ -241,7 +249,7 @@ ATLAS_API atlas_status_t atlas_paged_gqa_append_decode(
  * atlas_paged_gqa_decode plus num_kv_heads, head_dim, page_size and num_pages.
  * Every call shares the array: each call clears the counters and error word
  * on its stream before the launch, and calls that overlap on the GPU race.
- * When the split-KV partials of the balanced partition would not fit, the
+ * When the split-KV partials of the automatic partition would not fit, the
  * call runs one CTA per segment (no partials); a call that would then need a
  * segment longer than 65536 tokens returns ATLAS_ERR_WORKSPACE.  The first
  * call on a device looks up the array's address with that device current;

@@ -30,6 +30,7 @@ DEVERR_TIMEOUT = 0x8
 OPT_SPLIT_TOKENS = 1
 OPT_STAGES = 2
 OPT_WAVES = 3
+OPT_PARTITION = 4
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 

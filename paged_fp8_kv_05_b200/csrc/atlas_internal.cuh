@@ -48,7 +48,8 @@ struct DecodeParams {
   int row_blocks;
   int max_units;              // most 32-token units one CTA is given
   int max_portions;           // most segments one CTA's range meets
-  int per_segment;            // 1: CTA c = segment c (no partials); 0: balanced ranges
+  int grid_mode;              // 1: grid partition (CTA = split of a segment), 0: balanced
+  int num_splits, split_tokens;  // grid partition
   float qk_scale_log2;        // sm_scale * log2(e); k_scale[h] is folded in per head
   // fused append (A0): when k_new != nullptr the kernel first quantises and
   // writes the q_len new tokens of each sequence, positions L - q_len .. L - 1
@@ -61,20 +62,29 @@ cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t s
 
 // Launch shape of the decode kernel for one call (A1).  A segment is
 // (sequence, KV head, row group of rows_per_cta query rows); a unit is 32 KV
-// tokens of a segment.  Balanced mode: the units of all segments, in (b, h, rg)
-// order, are cut into `grid` equal ranges, one per CTA; a segment cut by a
-// range boundary leaves one partial per CTA it meets, merged by the CTA that
-// finishes it last.  Per-segment mode: one CTA per segment, no partials.
+// tokens of a segment.
+//  * Grid partition: CTA = one split of split_tokens tokens of one segment
+//    (num_splits per segment, as if every sequence were max_seq_len long;
+//    splits past a sequence's end exit at once).  The hardware hands CTAs to
+//    SMs as they free up, which evens out SMs that get slower memory service.
+//  * Balanced partition: the units of all segments, in (b, h, rg) order, are
+//    cut into `grid` equal ranges, one per CTA, whatever the length mix.
+// Either way a segment cut in several parts leaves one partial per part,
+// merged by log-sum-exp by the CTA that finishes the segment last.
+enum { kPartitionAuto = 0, kPartitionGrid = 1, kPartitionBalanced = 2 };
+
 struct DecodeLaunch {
   int rows_per_warp, rbg, rows_per_cta, row_blocks, stages;
   int waves;             // automatic grid: this many CTAs per resident CTA slot
+  int grid_mode;         // 1: grid partition, 0: balanced
+  int split_tokens;      // grid partition: tokens per split (a multiple of 64)
+  int num_splits;        // grid partition: splits per segment
   long long segs;        // B * Hkv * row_blocks
   long long units_max;   // segs * ceil(max_seq_len / 32): units if every L were max_seq_len
   long long grid;        // CTAs
   int max_units;         // units of the largest range
   int max_portions;      // segments the largest range can meet
-  int per_segment;
-  long long slots;       // partial slots: segs + grid (0 in per-segment mode)
+  long long slots;       // partial slots (0: no segment is ever cut)
 };
 
 constexpr int kMaxUnitsPerCta = 1024;  // bounds the per-CTA unit table in shared memory
@@ -84,10 +94,13 @@ inline int decode_target_occupancy(int rows_per_warp, int rbg) {
   return (rows_per_warp <= 8 && rbg == 1) ? 3 : 2;
 }
 
-// split_tokens > 0: ranges of about split_tokens KV tokens (a multiple of 32);
-// 0: `waves` ranges per resident CTA slot of the GPU (waves >= 1).
+// split_tokens > 0: splits / ranges of about split_tokens KV tokens; 0: the
+// automatic choice.  partition: kPartition*.  Automatic: the balanced
+// partition when one K/V stream serves the whole CTA (rbg 4: no in-CTA
+// combine, so range portions switch cheaply, and ragged lengths balance),
+// the grid partition otherwise.
 inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_len, int sms,
-                                int split_tokens, int stages_override, bool per_segment,
+                                int split_tokens, int stages_override, int partition,
                                 int waves = 1) {
   DecodeLaunch L;
   L.waves = waves < 1 ? 1 : waves;
@@ -101,12 +114,30 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
   L.segs = (long long)B * Hkv * L.row_blocks;
   const long long seg_units = ((long long)max_seq_len + 31) / 32;
   L.units_max = L.segs * seg_units;
-  L.per_segment = per_segment ? 1 : 0;
-  if (per_segment) {
-    L.grid = L.segs;
-    L.max_units = (int)(seg_units < 1 ? 1 : (seg_units > 0x7FFFFFFF ? 0x7FFFFFFF : seg_units));
+  const long long resident = (long long)sms * decode_target_occupancy(L.rows_per_warp, L.rbg);
+  L.grid_mode = (partition == kPartitionGrid || (partition == kPartitionAuto && L.rbg != 4));
+  if (L.grid_mode) {
+    long long T;
+    if (split_tokens > 0) {
+      T = (split_tokens + 63) / 64 * 64;
+    } else {
+      // about `waves` waves of resident CTAs if every sequence were max_seq_len
+      // long: splits a multiple of 64 tokens in [256, 8192]
+      const long long segs = L.segs > 0 ? L.segs : 1;
+      long long want = (resident * L.waves + segs - 1) / segs;
+      if (want < 1) want = 1;
+      T = ((long long)max_seq_len + want - 1) / want;
+      T = (T + 63) / 64 * 64;
+      if (T < 256) T = 256;
+      if (T > 8192) T = 8192;
+    }
+    L.split_tokens = (int)T;
+    L.num_splits = (int)(((long long)max_seq_len + T - 1) / T);
+    if (L.num_splits < 1) L.num_splits = 1;
+    L.grid = L.segs * L.num_splits;
+    L.max_units = (int)((T + 31) / 32);
     L.max_portions = 1;
-    L.slots = 0;
+    L.slots = L.num_splits > 1 ? L.segs * L.num_splits : 0;
     return L;
   }
   long long g;
@@ -114,7 +145,7 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
     const long long per = (split_tokens + 31) / 32;
     g = (L.units_max + per - 1) / per;
   } else {
-    g = (long long)sms * decode_target_occupancy(L.rows_per_warp, L.rbg) * L.waves;
+    g = resident * L.waves;
   }
   if (g > L.units_max) g = L.units_max;
   if (g < 1) g = 1;
@@ -127,6 +158,8 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
   L.max_units = (int)(mu < 1 ? 1 : mu);
   L.max_portions = (int)(L.segs < L.max_units ? L.segs : L.max_units);
   L.slots = L.segs + g;
+  L.split_tokens = 32 * L.max_units;
+  L.num_splits = 0;
   return L;
 }
 
@@ -140,7 +173,7 @@ cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg,
 size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units,
                              int max_portions);
 
-// Balanced mode without a split override: lower L.grid (and raise
+// Balanced partition without a split override: lower L.grid (and raise
 // L.max_units) until the CTAs fill L.waves waves of resident CTAs on `sms`
 // SMs, as far as the shared-memory footprint allows.  Needs a current CUDA device; leaves L alone
 // if the occupancy query fails.

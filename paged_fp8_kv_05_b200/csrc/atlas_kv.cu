@@ -20,6 +20,7 @@ struct atlas_kv_pool {
   int32_t split_override;
   int32_t stages_override;
   int32_t waves_override;
+  int32_t partition_override;
   size_t counters_bytes;  // largest counter block any accepted call uses
 };
 
@@ -66,18 +67,18 @@ WsLayout ws_layout(const atlas::DecodeLaunch& L, int head_dim) {
   return w;
 }
 
-// Split-KV partition (A1): balanced ranges of 32-token units, one per resident
-// CTA slot, or ranges of about split_override tokens when one is set.  The
-// range length adapts to the lengths and the SM count -- the "block size
-// adapted to sequence length and architecture" of the Atlas deep-dive's
-// attention paragraph, taken to equal work per CTA.
+// Split-KV partition (A1): splits of each segment handed to SMs by the
+// hardware, or balanced ranges of 32-token units (see atlas::plan_decode).
+// The split / range length adapts to the lengths and the SM count -- the
+// "block size adapted to sequence length and architecture" of the Atlas
+// deep-dive's attention paragraph.
 atlas::DecodeLaunch make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
                               int max_seq_len, int sms, bool fit) {
   atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, pool->num_kv_heads, q_len,
                                              max_seq_len, sms, pool->split_override,
-                                             pool->stages_override, false,
+                                             pool->stages_override, pool->partition_override,
                                              pool->waves_override > 0 ? pool->waves_override : 1);
-  if (fit && pool->split_override == 0) {
+  if (fit && pool->split_override == 0 && !L.grid_mode) {
     const int R = q_len * (num_q_heads / pool->num_kv_heads);
     atlas::decode_fp8_fit_grid(pool->head_dim, R < L.rows_per_cta ? R : L.rows_per_cta, sms, L);
   }
@@ -123,13 +124,15 @@ size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t nu
   size_t need = 0;
   for (int ql = 1; ql <= max_q_len; ++ql) {
     const int msl = max_seq_len > ql ? max_seq_len : ql;
-    // the automatic plan, and the finest split override the caller will set
-    for (int split : {0, min_split_tokens}) {
-      const atlas::DecodeLaunch L =
-          atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, msl, sms, split, 0, false);
-      const size_t t = ws_layout(L, head_dim).total;
-      if (t > need) need = t;
-    }
+    // both partitions, automatic and with the finest split override the caller
+    // will set
+    for (int part : {atlas::kPartitionGrid, atlas::kPartitionBalanced})
+      for (int split : {0, min_split_tokens}) {
+        const atlas::DecodeLaunch L =
+            atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, msl, sms, split, 0, part);
+        const size_t t = ws_layout(L, head_dim).total;
+        if (t > need) need = t;
+      }
   }
   return need;
 }
@@ -152,7 +155,7 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   size_t counters_bytes = 0;
   for (int ql = 1; ql <= max_q_len; ++ql) {
     const atlas::DecodeLaunch L = atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, ql,
-                                                     kDefaultSms, 0, 0, false);
+                                                     kDefaultSms, 0, 0, atlas::kPartitionAuto);
     const size_t c = align_up((size_t)L.segs * sizeof(int32_t), kAlign);
     if (c > counters_bytes) counters_bytes = c;
   }
@@ -175,6 +178,7 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   p->split_override = 0;
   p->stages_override = 0;
   p->waves_override = 0;
+  p->partition_override = 0;
   p->counters_bytes = counters_bytes;
   *out = p;
   return ATLAS_OK;
@@ -206,6 +210,10 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
     case ATLAS_OPT_WAVES:
       if (value < 0 || value > 8) return ATLAS_ERR_INVALID_ARG;
       pool->waves_override = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_PARTITION:
+      if (value < 0 || value > 2) return ATLAS_ERR_INVALID_ARG;
+      pool->partition_override = value;
       return ATLAS_OK;
   }
   return ATLAS_ERR_INVALID_ARG;
@@ -263,12 +271,15 @@ atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t 
   const bool dev = device_present();
   const int sms = dev ? device_sm_count() : kDefaultSms;
   const atlas::DecodeLaunch L = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, dev);
-  const long long seg_units = ((long long)max_seq_len + 31) / 32;
-  long long spread = 1 + (seg_units - 1 + L.max_units - 1) / L.max_units;
-  if (spread > L.grid) spread = L.grid;
-  const int32_t split = pool->split_override > 0 ? pool->split_override : 32 * L.max_units;
-  const int32_t f[ATLAS_PLAN_FIELDS] = {split, (int32_t)spread, 1, L.rows_per_cta,
-                                        L.row_blocks, 1,
+  long long spread = L.num_splits;  // grid partition: splits per segment
+  if (!L.grid_mode) {  // balanced: most ranges a max-length segment can meet
+    const long long seg_units = ((long long)max_seq_len + 31) / 32;
+    spread = 1 + (seg_units - 1 + L.max_units - 1) / L.max_units;
+    if (spread > L.grid) spread = L.grid;
+  }
+  const int32_t split = pool->split_override > 0 ? pool->split_override : L.split_tokens;
+  const int32_t f[ATLAS_PLAN_FIELDS] = {split, (int32_t)spread, L.grid_mode ? 1 : 2,
+                                        L.rows_per_cta, L.row_blocks, 1,
                                         (int32_t)(L.grid > 0x7FFFFFFF ? 0x7FFFFFFF : L.grid)};
   for (int i = 0; i < n && i < ATLAS_PLAN_FIELDS; ++i) plan[i] = f[i];
   return ATLAS_OK;
@@ -329,7 +340,9 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.row_blocks = L.row_blocks;
   p.max_units = L.max_units;
   p.max_portions = L.max_portions;
-  p.per_segment = 0;
+  p.grid_mode = L.grid_mode;
+  p.num_splits = L.num_splits;
+  p.split_tokens = L.split_tokens;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)pool->head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
   p.k_new = k_new;

@@ -165,7 +165,8 @@ struct Portion {
   int L;                // the sequence's length
   int ua;               // first unit of the portion inside the segment
   int k0;               // first unit of the portion inside the CTA's range
-  int c_first, c_last;  // first and last CTA that hold part of the segment
+  int slot0;            // first partial slot of the segment
+  int my, n_parts;      // this portion's part index and the segment's part count
   float k_scale, v_scale;  // the KV head's dequantisation scales
 };
 
@@ -281,20 +282,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 
   // ---- this CTA's range of units and its portions (A1)
   long long u0 = 0, u1 = 0;
-  if (p.per_segment) {
-    // CTA cid is segment cid: the whole segment, one portion, no partial
-    const int b = cid / Hs, seg = cid % Hs;
+  if (p.grid_mode) {
+    // CTA cid is split (cid % num_splits) of segment (cid / num_splits): tokens
+    // [split * T, split * T + T) of it, one portion; a sequence split in n_parts
+    // leaves n_parts partials (slots segment * num_splits + split)
+    const int split = cid % p.num_splits, sg = cid / p.num_splits;
+    const int b = sg / Hs, seg = sg % Hs;
     const int L = __ldg(p.seq_lens + b);
-    if (!valid_len(L)) return;  // CTA-uniform
+    if (!valid_len(L)) return;  // CTA-uniform; its rows were zeroed above
+    const int t_begin = split * p.split_tokens;
+    if (t_begin >= L) return;
     if (tid == 0) {
       Portion P;
-      P.b = b; P.seg = seg; P.L = L; P.ua = 0; P.k0 = 0; P.c_first = P.c_last = cid;
+      P.b = b; P.seg = seg; P.L = L; P.ua = t_begin / kUnit; P.k0 = 0;
+      P.slot0 = sg * p.num_splits;
+      P.my = split;
+      P.n_parts = (L + p.split_tokens - 1) / p.split_tokens;
       P.k_scale = __ldg(p.k_scale + seg / RB);
       P.v_scale = __ldg(p.v_scale + seg / RB);
       s_port[0] = P;
       s_nport = 1;
     }
-    u1 = units_of(L);
+    u1 = units_of(min(L - t_begin, p.split_tokens));
   } else {
     // every thread takes a contiguous run of sequences; a block-wide exclusive
     // scan of the runs' unit counts gives each run's first global unit
@@ -357,8 +366,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
             Q.b = bb; Q.seg = seg; Q.L = L;
             Q.ua = (int)(a - s0);
             Q.k0 = (int)(a - u0);
-            Q.c_first = owner_cta(s0, U, Ge);
-            Q.c_last = owner_cta(s0 + n - 1, U, Ge);
+            const int c_first = owner_cta(s0, U, Ge);
+            Q.slot0 = (bb * Hs + seg) + c_first;
+            Q.my = cid - c_first;
+            Q.n_parts = owner_cta(s0 + n - 1, U, Ge) - c_first + 1;
             Q.k_scale = __ldg(p.k_scale + seg / RB);
             Q.v_scale = __ldg(p.v_scale + seg / RB);
             s_port[slot_out++] = Q;
@@ -710,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const int rows_cta = min(RC, Rtot - cta_row0);
     const int row0 = cta_row0 + rbw * RW;  // this warp's first row
     const int kb = P.k0, ke = port_end(pi);
-    const bool whole = (P.c_first == P.c_last);
+    const bool whole = (P.n_parts == 1);
     if (!whole) {
       if (n_cut == 0) cut0 = pi; else cut1 = pi;
       n_cut = min(n_cut + 1, 2);
@@ -863,11 +874,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         l_full[nt][e] = l;
       }
 
-    // ---- where the portion's result goes: the output, or partial slot
-    // (segment + CTA) when other CTAs hold parts of the segment
-    const int seg_idx = b * Hs + seg;
+    // ---- where the portion's result goes: the output, or the partial slot of
+    // this part when other CTAs hold the segment's other parts
     const float vs = P.v_scale;
-    const size_t slot = (size_t)seg_idx + cid;
+    const size_t slot = (size_t)P.slot0 + P.my;
 
     if constexpr (NSTREAM == 1) {
       // one stream: every warp owns its rows outright; store from registers
@@ -979,12 +989,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const int rows_cta = min(RC, Rtot - cta_row0);
     int32_t* counter = p.counters + seg_idx;
     __syncthreads();  // every thread's partial stores are fenced; s_is_last is free
-    if (tid == 0) s_is_last = (atomicAdd(counter, 1) == P.c_last - P.c_first);
+    if (tid == 0) s_is_last = (atomicAdd(counter, 1) == P.n_parts - 1);
     __syncthreads();
     if (!s_is_last) continue;
     __threadfence();
-    const size_t s0 = (size_t)seg_idx + P.c_first;
-    const int n_slots = P.c_last - P.c_first + 1;
+    const size_t s0 = (size_t)P.slot0;
+    const int n_slots = P.n_parts;
     // per row: reference M and denominator over the slots' log2-sum-exp values
     for (int lr = tid; lr < rows_cta; lr += kThreads) {
       float M = -INFINITY, den = 0.f;
@@ -1070,7 +1080,7 @@ size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units
 }
 
 void decode_fp8_fit_grid(int D, int rows, int sms, DecodeLaunch& L) {
-  if (L.per_segment) return;
+  if (L.grid_mode) return;
   for (int it = 0; it < 4; ++it) {
     const size_t smem = decode_fp8_smem_bytes(D, L.stages, L.rbg, rows, L.max_units,
                                               L.max_portions);

@@ -87,11 +87,11 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   }
   const int R = q_len * (num_q_heads / num_kv_heads);
 
-  // the balanced partition of the pool-based entry point if its scratch --
+  // the automatic partition of the pool-based entry point if its scratch --
   // [error word][counters][log2-sum-exp][O partials] -- fits; else one CTA per
-  // segment, which needs only the error word
+  // segment (grid partition with a single split), which writes no partials
   atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len,
-                                             max_seq_len, sms, 0, 0, false);
+                                             max_seq_len, sms, 0, 0, atlas::kPartitionAuto);
   atlas::decode_fp8_fit_grid(head_dim, R < L.rows_per_cta ? R : L.rows_per_cta, sms, L);
   size_t counters_off = kAlign;
   size_t lse_off = counters_off + align_up((size_t)L.segs * sizeof(int32_t), kAlign);
@@ -99,9 +99,11 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   size_t o_off = lse_off + align_up(rows * sizeof(float), kAlign);
   size_t clear = lse_off;  // error word + counters
   if (o_off + rows * head_dim * sizeof(float) > kScratchBytes) {
-    L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len, max_seq_len, sms, 0, 0, true);
+    const int whole = (int)(((long long)max_seq_len + 63) / 64 * 64);
     // one segment's unit table lives in shared memory: bound its length
-    if (L.max_units > 2 * atlas::kMaxUnitsPerCta) return ATLAS_ERR_WORKSPACE;
+    if (whole > 64 * atlas::kMaxUnitsPerCta) return ATLAS_ERR_WORKSPACE;
+    L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len, max_seq_len, sms, whole, 0,
+                           atlas::kPartitionGrid);
     lse_off = o_off = counters_off;
     clear = kAlign;
   }
@@ -138,7 +140,9 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   p.row_blocks = L.row_blocks;
   p.max_units = L.max_units;
   p.max_portions = L.max_portions;
-  p.per_segment = L.per_segment;
+  p.grid_mode = L.grid_mode;
+  p.num_splits = L.num_splits;
+  p.split_tokens = L.split_tokens;
   const double scale = sm_scale > 0.f ? (double)sm_scale : 1.0 / sqrt((double)head_dim);
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
   p.k_new = nullptr;  // decode only

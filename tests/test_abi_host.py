@@ -113,16 +113,25 @@ def test_pool_create_ok_and_plan_is_host_only():
         buf = (ctypes.c_int32 * 7)()
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 100, buf, 7) == ak.ATLAS_OK
         plan = dict(zip(ak.PLAN_FIELDS, buf))
-        # 2 x 2 segments of 4 units (100 tokens): 16 units, one per CTA
-        assert plan["split_tokens"] == 32 and plan["num_splits"] == 4
-        assert plan["grid_ctas"] == 16
+        # grid partition: 2 x 2 segments of 4 rows, one split of 256 tokens each
+        # (the smallest automatic split) for max_seq_len 100
+        assert plan["kernel"] == 1 and plan["split_tokens"] == 256 and plan["num_splits"] == 1
+        assert plan["grid_ctas"] == 4
         assert plan["rows_per_cta"] == 4 and plan["row_blocks"] == 1 and plan["launches"] == 1
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 5, 100, buf, 7) == ak.ATLAS_OK
         assert buf[3] == 32 and buf[4] == 1           # 5 x 4 rows: two warps of 16 share K/V
         assert ak._lib.atlas_kv_pool_set_split_tokens(h, 128) == ak.ATLAS_OK
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 1000, buf, 7) == ak.ATLAS_OK
-        # 4 segments x 32 units in ranges of 4 units: 32 CTAs; a segment meets <= 9
-        assert buf[0] == 128 and buf[1] == 9 and buf[6] == 32
+        # grid: 1000 tokens in splits of 128 -> 8 splits x 4 segments
+        assert buf[0] == 128 and buf[1] == 8 and buf[2] == 1 and buf[6] == 32
+        # balanced: 4 segments x 32 units in ranges of 4 units: 32 CTAs; a
+        # segment meets at most 9 of them
+        assert ak._lib.atlas_kv_pool_set_option(h, ak.OPT_PARTITION, 2) == ak.ATLAS_OK
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 1, 1000, buf, 7) == ak.ATLAS_OK
+        assert buf[0] == 128 and buf[1] == 9 and buf[2] == 2 and buf[6] == 32
+        for bad in (-1, 3):
+            assert ak._lib.atlas_kv_pool_set_option(h, ak.OPT_PARTITION, bad) == ak.ATLAS_ERR_INVALID_ARG
+        assert ak._lib.atlas_kv_pool_set_option(h, ak.OPT_PARTITION, 0) == ak.ATLAS_OK
         for bad in (-64, 32, 100, 16384):
             assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
         for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 2, 0), (ak.OPT_STAGES, 0, 0),

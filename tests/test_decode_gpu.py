@@ -27,14 +27,26 @@ def _dw(w, **kw):
     return DeviceWorkload(w, **kw)
 
 
-@pytest.mark.parametrize("cfg", [0, 1, 2, 4])
-def test_named_workload_full_output(ak, cfg):
+_ORACLE = {}
+
+
+def _oracle_named(cfg, w):
+    if cfg not in _ORACLE:
+        _ORACLE[cfg] = oracle_decode(w)
+    return _ORACLE[cfg]
+
+
+# partition 0 = automatic (grid for 0-2, balanced for the MQA case 4); the
+# other partition of configs 1 and 4 is checked too
+@pytest.mark.parametrize("cfg,partition", [(0, 0), (1, 0), (2, 0), (4, 0), (1, 2), (4, 1)])
+def test_named_workload_full_output(ak, cfg, partition):
     w = workloads.config_workload(cfg)
     dw = _dw(w)
+    dw.pool.set_option(ak.OPT_PARTITION, partition)
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
-    ref = oracle_decode(w)
-    max_abs, rel = assert_close(got, ref, f"config {cfg}")
+    ref = _oracle_named(cfg, w)
+    max_abs, rel = assert_close(got, ref, f"config {cfg}, partition {partition}")
     print(f"config {cfg}: max-abs {max_abs:.3e} rel-L2 {rel:.3e} plan {dw.plan()}")
 
 
@@ -81,6 +93,28 @@ def test_edge_cases(ak, case):
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
     assert_close(got, oracle_decode(w), f"edge {case}")
+
+
+@pytest.mark.parametrize("partition", [1, 2])
+@pytest.mark.parametrize("split", [0, 64])
+@pytest.mark.parametrize("case", [
+    (4, 8, 2, 128, 16, [17, 31, 32, 33], 1),
+    (6, 32, 8, 128, 16, [1, 40, 900, 2000, 33, 64], 1),
+    (3, 40, 8, 128, 16, [5, 6, 210], 5),
+    (3, 64, 1, 128, 64, [64, 200, 1500], 1),
+])
+def test_both_partitions(ak, case, split, partition):
+    """Grid splits and balanced ranges, with automatic and 64-token parts (a
+    segment cut into many parts, merged by the CTA that finishes it last)."""
+    w = _case(*case, seed=11)
+    dw = _dw(w, min_split_tokens=64)
+    dw.pool.set_option(ak.OPT_PARTITION, partition)
+    dw.pool.set_split_tokens(split)
+    plan = dw.plan()
+    assert plan["kernel"] == partition
+    got = dw.decode().float().cpu().numpy()
+    assert dw.pool.device_error() == 0
+    assert_close(got, oracle_decode(w), f"{case} split {split} partition {partition}")
 
 
 @pytest.mark.parametrize("split", [64, 128, 192, 512, 8192])
