@@ -161,6 +161,10 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
                                      /* schedules them), 2 = balanced (equal ranges of   */
                                      /* 32-token units per CTA); auto takes balanced     */
                                      /* only when one K/V stream serves a whole CTA      */
+#define ATLAS_OPT_ROWS_PER_CTA   5   /* query rows one CTA serves: 0 = auto (the fewest */
+                                     /* of 4, 8, 16, 32, 64 holding q_len * G), else one */
+                                     /* of those; fewer rows make more row blocks, each  */
+                                     /* streaming the KV head's pages again              */
 
 /*
  * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of

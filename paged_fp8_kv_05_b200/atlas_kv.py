@@ -31,6 +31,7 @@ OPT_SPLIT_TOKENS = 1
 OPT_STAGES = 2
 OPT_WAVES = 3
 OPT_PARTITION = 4
+OPT_ROWS_PER_CTA = 5
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 

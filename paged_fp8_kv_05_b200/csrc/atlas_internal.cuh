@@ -99,15 +99,18 @@ inline int decode_target_occupancy(int rows_per_warp, int rbg) {
 // partition when one K/V stream serves the whole CTA (rbg 4: no in-CTA
 // combine, so range portions switch cheaply, and ragged lengths balance),
 // the grid partition otherwise.
+// rows_per_cta: 0 = automatic (the smallest of 4, 8, 16, 32, 64 that holds
+// all q_len * G rows of a KV head), else one of those (more row blocks).
 inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_len, int sms,
                                 int split_tokens, int stages_override, int partition,
-                                int waves = 1) {
+                                int waves = 1, int rows_per_cta = 0) {
   DecodeLaunch L;
   L.waves = waves < 1 ? 1 : waves;
   const int G = Hq / Hkv;
   const int R = q_len * G;
-  L.rows_per_warp = (R <= 4) ? 4 : (R <= 8) ? 8 : 16;  // 4: hi | lo packed MMA columns
-  L.rbg = (R <= 16) ? 1 : (R <= 32 ? 2 : 4);
+  const int rc = rows_per_cta > 0 ? rows_per_cta : (R <= 4 ? 4 : R <= 8 ? 8 : R <= 16 ? 16 : R <= 32 ? 32 : 64);
+  L.rows_per_warp = rc <= 8 ? rc : 16;  // 4: hi | lo packed MMA columns
+  L.rbg = rc <= 16 ? 1 : rc / 16;        // warps sharing one K/V stream
   L.rows_per_cta = L.rows_per_warp * L.rbg;
   L.row_blocks = (R + L.rows_per_cta - 1) / L.rows_per_cta;
   L.stages = stages_override > 0 ? stages_override : (L.rbg == 1 ? 2 : 3);
@@ -121,13 +124,21 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
     if (split_tokens > 0) {
       T = (split_tokens + 63) / 64 * 64;
     } else {
-      // about `waves` waves of resident CTAs if every sequence were max_seq_len
-      // long: splits a multiple of 64 tokens in [256, 8192]
+      // splits for n waves of resident CTAs if every sequence were max_seq_len
+      // long, a multiple of 64 tokens.  Two waves let the hardware even out
+      // the SMs, but a split under 2048 tokens spends too much of its time in
+      // the prologue -- unless even one wave needs shorter splits.  [256, 8192].
       const long long segs = L.segs > 0 ? L.segs : 1;
-      long long want = (resident * L.waves + segs - 1) / segs;
-      if (want < 1) want = 1;
-      T = ((long long)max_seq_len + want - 1) / want;
-      T = (T + 63) / 64 * 64;
+      auto split_for = [&](long long ctas) {
+        long long want = (ctas + segs - 1) / segs;
+        if (want < 1) want = 1;
+        const long long t = ((long long)max_seq_len + want - 1) / want;
+        return (t + 63) / 64 * 64;
+      };
+      const long long one_wave = split_for(resident * L.waves);
+      T = split_for(2 * resident * L.waves);
+      const long long lo = one_wave < 2048 ? one_wave : 2048;
+      if (T < lo) T = lo;
       if (T < 256) T = 256;
       if (T > 8192) T = 8192;
     }

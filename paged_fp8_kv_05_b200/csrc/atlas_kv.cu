@@ -21,6 +21,7 @@ struct atlas_kv_pool {
   int32_t stages_override;
   int32_t waves_override;
   int32_t partition_override;
+  int32_t rows_override;
   size_t counters_bytes;  // largest counter block any accepted call uses
 };
 
@@ -77,7 +78,8 @@ atlas::DecodeLaunch make_plan(const atlas_kv_pool* pool, int batch, int num_q_he
   atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, pool->num_kv_heads, q_len,
                                              max_seq_len, sms, pool->split_override,
                                              pool->stages_override, pool->partition_override,
-                                             pool->waves_override > 0 ? pool->waves_override : 1);
+                                             pool->waves_override > 0 ? pool->waves_override : 1,
+                                             pool->rows_override);
   if (fit && pool->split_override == 0 && !L.grid_mode) {
     const int R = q_len * (num_q_heads / pool->num_kv_heads);
     atlas::decode_fp8_fit_grid(pool->head_dim, R < L.rows_per_cta ? R : L.rows_per_cta, sms, L);
@@ -133,6 +135,11 @@ size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t nu
         const size_t t = ws_layout(L, head_dim).total;
         if (t > need) need = t;
       }
+    // the counter block of the finest row grouping (4 rows per block)
+    const atlas::DecodeLaunch L4 = atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql,
+                                                      msl, sms, 0, 0, atlas::kPartitionGrid, 1, 4);
+    const size_t c4 = kAlign + align_up((size_t)L4.segs * sizeof(int32_t), kAlign);
+    if (c4 > need) need = c4;
   }
   return need;
 }
@@ -154,8 +161,10 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
     return ATLAS_ERR_INVALID_ARG;
   size_t counters_bytes = 0;
   for (int ql = 1; ql <= max_q_len; ++ql) {
+    // the most segments any row grouping makes: 4 rows per block
     const atlas::DecodeLaunch L = atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql, ql,
-                                                     kDefaultSms, 0, 0, atlas::kPartitionAuto);
+                                                     kDefaultSms, 0, 0, atlas::kPartitionAuto, 1,
+                                                     4);
     const size_t c = align_up((size_t)L.segs * sizeof(int32_t), kAlign);
     if (c > counters_bytes) counters_bytes = c;
   }
@@ -179,6 +188,7 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   p->stages_override = 0;
   p->waves_override = 0;
   p->partition_override = 0;
+  p->rows_override = 0;
   p->counters_bytes = counters_bytes;
   *out = p;
   return ATLAS_OK;
@@ -214,6 +224,11 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
     case ATLAS_OPT_PARTITION:
       if (value < 0 || value > 2) return ATLAS_ERR_INVALID_ARG;
       pool->partition_override = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_ROWS_PER_CTA:
+      if (value != 0 && value != 4 && value != 8 && value != 16 && value != 32 && value != 64)
+        return ATLAS_ERR_INVALID_ARG;
+      pool->rows_override = value;
       return ATLAS_OK;
   }
   return ATLAS_ERR_INVALID_ARG;
