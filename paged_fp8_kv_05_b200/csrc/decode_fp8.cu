@@ -283,10 +283,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   // ---- this CTA's range of units and its portions (A1)
   long long u0 = 0, u1 = 0;
   if (p.grid_mode) {
-    // CTA cid is split (cid % num_splits) of segment (cid / num_splits): tokens
+    // CTA cid is split (cid / segs) of segment (cid % segs): tokens
     // [split * T, split * T + T) of it, one portion; a sequence split in n_parts
-    // leaves n_parts partials (slots segment * num_splits + split)
-    const int split = cid % p.num_splits, sg = cid / p.num_splits;
+    // leaves n_parts partials (slots segment * num_splits + split).  Split-major
+    // order: the first splits, full length for every long sequence, are handed
+    // out first, the shorter or empty last splits fill in behind them.
+    const int n_sg = G / p.num_splits;
+    const int split = cid / n_sg, sg = cid % n_sg;
     const int b = sg / Hs, seg = sg % Hs;
     const int L = __ldg(p.seq_lens + b);
     if (!valid_len(L)) return;  // CTA-uniform; its rows were zeroed above
