@@ -1,10 +1,9 @@
 // Internal declarations shared by the kernels and the C-ABI layer.
-// Device helpers here wrap single PTX instructions (conversion, warp MMA,
-// register-matrix transpose, base-2 exponential); none re-implements a
-// math-library routine.
+// Device helpers here wrap single PTX instructions (conversion,
+// register-matrix transpose, base-2 exponential, mbarriers, bulk copies); none
+// re-implements a math-library routine.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -124,10 +123,13 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
     if (split_tokens > 0) {
       T = (split_tokens + 63) / 64 * 64;
     } else {
-      // splits for n waves of resident CTAs if every sequence were max_seq_len
-      // long, a multiple of 64 tokens.  Two waves let the hardware even out
-      // the SMs, but a split under 2048 tokens spends too much of its time in
-      // the prologue -- unless even one wave needs shorter splits.  [256, 8192].
+      // splits for at least two waves of resident CTAs if every sequence were
+      // max_seq_len long (the split for two waves rounded down to a power of
+      // two: two to four waves), so that the hardware can even out the SMs;
+      // but a split under 2048 tokens spends too much of its time in the
+      // prologue -- unless even one wave needs shorter splits.  Multiple of
+      // 64 in [256, 8192].  (Measured on the long-context workload: 4096-token
+      // splits 148 µs, 4736: 160 µs, 3072: 167 µs; LLaMA-shaped: 2048 best.)
       const long long segs = L.segs > 0 ? L.segs : 1;
       auto split_for = [&](long long ctas) {
         long long want = (ctas + segs - 1) / segs;
@@ -136,7 +138,9 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
         return (t + 63) / 64 * 64;
       };
       const long long one_wave = split_for(resident * L.waves);
-      T = split_for(2 * resident * L.waves);
+      const long long two_waves = split_for(2 * resident * L.waves);
+      T = 64;
+      while (2 * T <= two_waves) T *= 2;
       const long long lo = one_wave < 2048 ? one_wave : 2048;
       if (T < lo) T = lo;
       if (T < 256) T = 256;
@@ -176,7 +180,7 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
 
 // FP8 tensor-core decode kernel.  rows_per_warp is 4, 8 or 16 and rbg (warps that
 // share one K/V stream) 1, 2 or 4; stages 2 or 3.  1-D grid of `grid` CTAs
-// (balanced ranges, or one per segment when p.per_segment).
+// (grid partition: segments x splits; balanced: one range each).
 cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
                               long long grid, cudaStream_t stream);
 
@@ -186,39 +190,19 @@ size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units
 
 // Balanced partition without a split override: lower L.grid (and raise
 // L.max_units) until the CTAs fill L.waves waves of resident CTAs on `sms`
-// SMs, as far as the shared-memory footprint allows.  Needs a current CUDA device; leaves L alone
-// if the occupancy query fails.
+// SMs, as far as the shared-memory footprint allows.  Needs a current CUDA
+// device; leaves L alone if the occupancy query fails.
 void decode_fp8_fit_grid(int D, int rows, int sms, DecodeLaunch& L);
 
 // ------------------------------------------------------------ device helpers
 
 #ifdef __CUDACC__
 
-// Two E4M3 codes (low byte first) -> f16x2 (exact: E4M3 is a subset of f16).
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 a, b;\n\t"
-      "mov.b32 {a, b}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
 // f16x2 with `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-// D += A * B, m16n8k16, f16 inputs, f32 accumulate.
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Transpose an 8x8 matrix of 16-bit elements held one b32 pair per thread.
@@ -232,22 +216,6 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 __device__ __forceinline__ float fast_exp2(float x) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
-// Streaming 16-byte / 8-byte read-only loads that skip L1 allocation.
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint2 ld_stream8(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(r.x), "=r"(r.y)
-               : "l"(p));
   return r;
 }
 
@@ -313,7 +281,7 @@ __device__ __forceinline__ void store16_v(uint8_t* v_pages, size_t head_page, in
   for (int k = 0; k < 16; ++k) dst[16 * k] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
 }
 
-// ---- shared-memory addresses, mbarriers and TMA (single PTX instructions)
+// ---- shared-memory addresses, mbarriers and bulk copies (single PTX instructions)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -326,10 +294,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Orders this thread's earlier global writes before later async-proxy reads.
@@ -385,16 +349,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// 2-D TMA tile load global -> shared, completion counted on `bar` (no multicast).
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
 

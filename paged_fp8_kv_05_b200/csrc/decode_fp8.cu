@@ -38,28 +38,32 @@
 // accumulator through movmatrix.trans, which hands each lane exactly those
 // four tokens of its row -- no shuffles.
 //
-// Work partition (persistent, balanced).  A segment is (sequence b, KV head h,
-// row group rg): ceil(L_b / 32) units of 32 KV tokens for up to RC query rows.
-// All units of all segments form one list (segments in (b, h, rg) order);
-// CTA c of the G CTAs takes units [c*U/G, (c+1)*U/G) of the U in the list, so
-// every CTA gets the same amount of KV to stream whatever the length mix (the
-// "block size adapted to sequence length" of the deep-dive, taken to its
-// limit).  Its range cuts the list into portions, one per segment it touches.
-// Its 4 warps form 4/RBG streams that take the CTA's units round-robin; the RBG
-// warps of a stream share one ring of S shared-memory stages, each holding the
-// K and V^T pieces of one unit (two 16-token page pieces, each a contiguous
-// block of 16*D bytes in its page), filled by 1-D bulk copies (cp.async.bulk,
-// no multicast) that complete on a "full" mbarrier; with RBG > 1 an "empty"
+// Work partition.  A segment is (sequence b, KV head h, row group rg):
+// ceil(L_b / 32) units of 32 KV tokens for up to RC query rows.  Two modes
+// share all code below the prologue:
+//  * grid: CTA = one split of split_tokens tokens of one segment; the hardware
+//    hands CTAs to SMs as slots free up (split-major order: first splits
+//    first);
+//  * balanced: all units of all segments form one list (segments in (b, h, rg)
+//    order) and CTA c of the G CTAs takes units [c*U/G, (c+1)*U/G), so every
+//    CTA streams the same amount of KV whatever the length mix; its range cuts
+//    the list into portions, one per segment it touches.
+// The "block size adapted to sequence length and architecture" of the Atlas
+// deep-dive is the host's choice of split length / range count.  The CTA's 4
+// warps form 4/RBG streams that take its units round-robin; the RBG warps of a
+// stream share one ring of S shared-memory stages, each holding the K and V^T
+// pieces of one unit (two 16-token page pieces, each a contiguous block of
+// 16*D bytes in its page), filled by 1-D bulk copies (cp.async.bulk, no
+// multicast) that complete on a "full" mbarrier; with RBG > 1 an "empty"
 // mbarrier counts the consumers before a stage is refilled.  The ring keeps
 // streaming across portion boundaries.  At the end of a portion the streams
-// combine their online-softmax states in shared memory; a segment that lies
-// inside one CTA is written out as bf16, otherwise the CTA writes
-// (O/l, log2-sum-exp) to the partial slot (segment + c) and the CTA that
-// finishes the segment last -- one atomic counter per segment, no waiting --
-// merges its slots and resets the counter.  A per-segment mode (CTA c = segment
-// c, no partials) serves callers with little scratch.  Every mbarrier wait is
-// bounded (200 ms of wall clock): a wait that runs out flags
-// ATLAS_DEVERR_TIMEOUT and the warp stops computing after draining its loads.
+// combine their online-softmax states in shared memory; a segment held by one
+// CTA is written out as bf16, otherwise the CTA writes (O/l, log2-sum-exp) to
+// its part's slot and the CTA that finishes the segment last -- one atomic
+// counter per segment, no waiting -- merges the parts and resets the counter.
+// Every mbarrier wait is bounded (200 ms of wall clock): a wait that runs out
+// flags ATLAS_DEVERR_TIMEOUT and the warp stops computing after draining its
+// loads.
 #include <float.h>
 #include <math.h>
 
