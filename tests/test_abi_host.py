@@ -212,3 +212,35 @@ def test_null_pool_is_rejected_everywhere():
     assert ak._lib.atlas_kv_pool_set_split_tokens(None, 0) == ak.ATLAS_ERR_INVALID_ARG
     assert ak._lib.atlas_kv_pool_destroy(None) == ak.ATLAS_OK
     assert _decode(None) == ak.ATLAS_ERR_INVALID_ARG
+
+
+def _plan_on_148_sms(B, Hq, Hkv, D, ps, q_len, max_seq_len, P=1024):
+    h = ctypes.c_void_p()
+    p = F.ptr
+    st = ak._lib.atlas_kv_pool_create(ctypes.byref(h), P, ps, Hkv, D, p, p, p, p, B, q_len, Hq,
+                                      p, ctypes.c_size_t(1 << 40))
+    assert st == ak.ATLAS_OK
+    try:
+        buf = (ctypes.c_int32 * 7)()
+        assert ak._lib.atlas_paged_gqa_decode_plan(h, B, Hq, q_len, max_seq_len, buf, 7) == 0
+        return dict(zip(ak.PLAN_FIELDS, buf))
+    finally:
+        ak._lib.atlas_kv_pool_destroy(h)
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="plans for a 148-SM part")
+@pytest.mark.parametrize("shape,want", [
+    # LLaMA-3-8B decode: 256 segments of 4 rows; two waves would need 1024-token
+    # splits, under the 2048-token floor that one wave allows -> 2048, 512 CTAs
+    ((32, 32, 8, 128, 16, 1, 4096), dict(kernel=1, split_tokens=2048, grid_ctas=512, rows_per_cta=4)),
+    # long context: 32 segments; two waves -> 4736 tokens, rounded down to 4096
+    ((4, 32, 8, 128, 16, 1, 131072), dict(kernel=1, split_tokens=4096, num_splits=32, grid_ctas=1024)),
+    # MTP verify: 1024 segments already fill the GPU; one split of the whole length
+    ((128, 40, 8, 128, 16, 5, 1152), dict(kernel=1, split_tokens=1152, grid_ctas=1024, rows_per_cta=32)),
+    # MQA with 64 rows: one K/V stream per CTA -> balanced ranges, 2 per SM
+    ((256, 64, 1, 128, 64, 1, 8192), dict(kernel=2, grid_ctas=296, rows_per_cta=64)),
+])
+def test_automatic_plan_of_the_named_shapes(shape, want):
+    plan = _plan_on_148_sms(*shape)
+    for k, v in want.items():
+        assert plan[k] == v, (k, plan)
