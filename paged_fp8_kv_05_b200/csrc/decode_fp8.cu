@@ -275,28 +275,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 
   // ---- invalid sequences (shorter than q_len, longer than the block-table row
   // or the host's max_seq_len): zero all their rows and flag them; one CTA per b
-  auto zero_invalid = [&]() {
-    for (int bb = cid; bb < p.B; bb += G) {
-      const int L = __ldg(p.seq_lens + bb);
-      if (valid_len(L)) continue;
-      if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
-      const size_t n = (size_t)p.q_len * p.Hq * D;
-      __nv_bfloat16* o = p.out + (size_t)bb * n;
-      for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
-    }
-  };
-  const int groups_per_page = p.ps / 16;
-  // index of 16-token piece `t` (a multiple of 16) of KV head h in blocks of
-  // 16*D bytes of the page arrays, or -1 past the end / for a bad page id
-  auto piece_index = [&](int pid, int t, int L, int h) {
-    if (t >= L) return -1;
-    if (pid < 0 || pid >= p.num_pages) {
-      atomicOr(p.err, ATLAS_DEVERR_PAGE_ID);
-      return -1;
-    }
-    const int pg = t / p.ps;
-    return (pid * p.Hkv + h) * groups_per_page + (t - pg * p.ps) / 16;
-  };
+  for (int bb = cid; bb < p.B; bb += G) {
+    const int L = __ldg(p.seq_lens + bb);
+    if (valid_len(L)) continue;
+    if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
+    const size_t n = (size_t)p.q_len * p.Hq * D;
+    __nv_bfloat16* o = p.out + (size_t)bb * n;
+    for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
+  }
 
   // ---- this CTA's range of units and its portions (A1)
   long long u0 = 0, u1 = 0;
@@ -308,55 +294,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     // out first, the shorter or empty last splits fill in behind them.
     const int n_sg = G / p.num_splits;
     const int split = cid / n_sg, sg = cid % n_sg;
-    const int b = sg / Hs, seg = sg % Hs, h = seg / RB;
-    const int t_begin = split * p.split_tokens;
-    // every independent load goes out first: the page ids of this thread's
-    // first two units (A2, before the length is known: the table row is read
-    // in bounds either way), the length and the scales
-    const int32_t* bt_row = p.block_table + (size_t)b * p.max_blocks;
-    const int max_tok = p.max_blocks * p.ps;
-    int pid[2][2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int t = t_begin + kUnit * (tid + kThreads * r) + 16 * half;
-        const bool in_split = kUnit * (tid + kThreads * r) < p.split_tokens;
-        pid[r][half] = (in_split && t < max_tok) ? __ldg(bt_row + t / p.ps) : -1;
-      }
+    const int b = sg / Hs, seg = sg % Hs;
     const int L = __ldg(p.seq_lens + b);
-    const float ksc = __ldg(p.k_scale + h), vsc = __ldg(p.v_scale + h);
-    zero_invalid();
-    if (!valid_len(L)) return;  // CTA-uniform; the sequence's rows are zeroed
+    if (!valid_len(L)) return;  // CTA-uniform; its rows were zeroed above
+    const int t_begin = split * p.split_tokens;
     if (t_begin >= L) return;
-    u1 = units_of(min(L - t_begin, p.split_tokens));
-    const int U_here = (int)u1;
-    for (int k = tid; k < U_here; k += kThreads) {
-      const int t0 = t_begin + kUnit * k;
-      int pa, pb;
-      if (k < 2 * kThreads) {
-        const bool second = k >= kThreads;
-        pa = second ? pid[1][0] : pid[0][0];
-        pb = second ? pid[1][1] : pid[0][1];
-      } else {  // splits longer than 2 * 128 units (one CTA per segment)
-        pa = __ldg(bt_row + t0 / p.ps);
-        pb = t0 + 16 < max_tok ? __ldg(bt_row + (t0 + 16) / p.ps) : -1;
-      }
-      s_pieces[k] = make_int2(piece_index(pa, t0, L, h), piece_index(pb, t0 + 16, L, h));
-    }
     if (tid == 0) {
       Portion P;
       P.b = b; P.seg = seg; P.L = L; P.ua = t_begin / kUnit; P.k0 = 0;
       P.slot0 = sg * p.num_splits;
       P.my = split;
       P.n_parts = (L + p.split_tokens - 1) / p.split_tokens;
-      P.k_scale = ksc;
-      P.v_scale = vsc;
+      P.k_scale = __ldg(p.k_scale + seg / RB);
+      P.v_scale = __ldg(p.v_scale + seg / RB);
       s_port[0] = P;
       s_nport = 1;
     }
+    u1 = units_of(min(L - t_begin, p.split_tokens));
   } else {
-    zero_invalid();
     // every thread takes a contiguous run of sequences; a block-wide exclusive
     // scan of the runs' unit counts gives each run's first global unit
     const int per = (p.B + kThreads - 1) / kThreads;
@@ -456,78 +411,38 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   prefetch_q(0);
   if (n_port > 1) prefetch_q(1);
 
-  // ---- A2, block-table gather (balanced partition; the grid partition did it
-  // above): the two 16-token pieces of unit k of the range, as indices of
-  // 16*D-byte blocks of the page arrays (-1: past the end of the sequence or a
-  // bad page id).  The divisions happen here, once.
-  auto portion_of = [&](int k) {  // last portion with k0 <= k
-    int lo = 0, hi = n_port - 1;
+  // ---- A2, block-table gather: the two 16-token pieces of unit k of the
+  // range, as indices of 16*D-byte blocks of the page arrays (-1: past the end
+  // of the sequence or a bad page id).  The divisions happen here, once.
+  const int groups_per_page = p.ps / 16;
+  auto build_piece = [&](int k) {
+    int lo = 0, hi = n_port - 1;   // last portion with k0 <= k
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_port[mid].k0 <= k) lo = mid; else hi = mid - 1;
     }
-    return lo;
+    const Portion P = s_port[lo];
+    const int h = P.seg / RB;
+    const int t0 = kUnit * (P.ua + k - P.k0);
+    int pc[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int t = t0 + 16 * half;
+      pc[half] = -1;
+      if (t < P.L) {
+        const int pg = t / p.ps;
+        const int pid = __ldg(p.block_table + (size_t)P.b * p.max_blocks + pg);
+        if (pid < 0 || pid >= p.num_pages)
+          atomicOr(p.err, ATLAS_DEVERR_PAGE_ID);
+        else
+          pc[half] = (pid * p.Hkv + h) * groups_per_page + (t - pg * p.ps) / 16;
+      }
+    }
+    s_pieces[k] = make_int2(pc[0], pc[1]);
   };
-  if (!p.grid_mode) {
-    for (int k = tid; k < U_cta; k += kThreads) {
-      const Portion P = s_port[portion_of(k)];
-      const int h = P.seg / RB;
-      const int t0 = kUnit * (P.ua + k - P.k0);
-      const int32_t* bt_row = p.block_table + (size_t)P.b * p.max_blocks;
-      const int pa = t0 < P.L ? __ldg(bt_row + t0 / p.ps) : -1;
-      const int pb = t0 + 16 < P.L ? __ldg(bt_row + (t0 + 16) / p.ps) : -1;
-      s_pieces[k] = make_int2(piece_index(pa, t0, P.L, h), piece_index(pb, t0 + 16, P.L, h));
-    }
-  }
-  if (tid < NSTREAM * S) {
-    mbar_init(&full_bar[tid], 1);
-    mbar_init(&empty_bar[tid], RBG);
-  }
-  if (tid == 0) fence_mbar_init();
-  // do the units the streams load first (k < NSTREAM * S) hold a token that
-  // the fused append writes?  If not, their loads go out before the append.
-  bool holds_new = false;
-  if (p.k_new != nullptr && tid < NSTREAM * S && tid < U_cta) {
-    const Portion P = s_port[portion_of(tid)];
-    holds_new = kUnit * (P.ua + tid - P.k0) + kUnit > P.L - p.q_len;
-  }
-  const bool late_issue = __syncthreads_or(holds_new);  // table and barriers ready
-
-  // this stream's units: k = stream + NSTREAM * i, i < n_my
-  const int n_my = (stream < U_cta) ? (U_cta - stream + NSTREAM - 1) / NSTREAM : 0;
-  const bool producer = (rbw == 0) && (lane == 0);
-  constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
-  auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
-    const int st = i % S;
-    uint64_t* bar = &full_bar[stream * S + st];
-    uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
-    const int2 pc = s_pieces[stream + NSTREAM * i];
-    const uint32_t bytes = (pc.x >= 0 ? 2 * TILE : 0) + (pc.y >= 0 ? 2 * TILE : 0);
-    if (bytes == 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    mbar_arrive_expect_tx(bar, bytes);
-    // a 16-token piece is TILE contiguous bytes in both layouts: K rows
-    // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
-    if (pc.x >= 0) {
-      bulk_load(dst, p.k_pages + (size_t)pc.x * kPiece, TILE, bar);
-      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pc.x * kPiece, TILE, bar);
-    }
-    if (pc.y >= 0) {
-      bulk_load(dst + TILE, p.k_pages + (size_t)pc.y * kPiece, TILE, bar);
-      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pc.y * kPiece, TILE, bar);
-    }
-  };
-  if (!late_issue && producer) {
-    for (int i = 0; i < S && i < n_my; ++i) issue(i);
-  }
-
   // ---- A0, fused append: the step's new tokens (positions L - q_len .. L - 1)
-  // that fall in this CTA's portions are quantised and stored, and made visible
-  // to the bulk copies (fences here, then a CTA barrier) before any copy that
-  // reads their pieces is queued: the first loads wait for it only if they
-  // hold such a piece; later refills come after the first portion's barrier
+  // that fall in this CTA's portions are quantised and stored first, while HBM
+  // is still idle, and made visible to the bulk copies before any is queued
   if (p.k_new != nullptr) {
     bool wrote = false;
     for (int pi = 0; pi < n_port; ++pi) {
@@ -567,11 +482,43 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       fence_proxy_async_global();
     }
   }
-  if (late_issue) {
-    __syncthreads();  // appended tokens visible to the bulk copies
-    if (producer) {
-      for (int i = 0; i < S && i < n_my; ++i) issue(i);
+  // the whole unit table, before any bulk copy is queued
+  for (int k = tid; k < U_cta; k += kThreads) build_piece(k);
+  if (tid < NSTREAM * S) {
+    mbar_init(&full_bar[tid], 1);
+    mbar_init(&empty_bar[tid], RBG);
+  }
+  if (tid == 0) fence_mbar_init();
+  __syncthreads();  // table, barriers and appended tokens ready
+
+  // this stream's units: k = stream + NSTREAM * i, i < n_my
+  const int n_my = (stream < U_cta) ? (U_cta - stream + NSTREAM - 1) / NSTREAM : 0;
+  const bool producer = (rbw == 0) && (lane == 0);
+  constexpr size_t kPiece = (size_t)16 * D;  // bytes of one 16-token piece
+  auto issue = [&](int i) {  // producer lane only: stage i % S <- unit i
+    const int st = i % S;
+    uint64_t* bar = &full_bar[stream * S + st];
+    uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
+    const int2 pc = s_pieces[stream + NSTREAM * i];
+    const uint32_t bytes = (pc.x >= 0 ? 2 * TILE : 0) + (pc.y >= 0 ? 2 * TILE : 0);
+    if (bytes == 0) {
+      mbar_arrive(bar);
+      return;
     }
+    mbar_arrive_expect_tx(bar, bytes);
+    // a 16-token piece is TILE contiguous bytes in both layouts: K rows
+    // (slot0 .. slot0 + 15) x D, and V group slot0 / 16 ([D][16])
+    if (pc.x >= 0) {
+      bulk_load(dst, p.k_pages + (size_t)pc.x * kPiece, TILE, bar);
+      bulk_load(dst + 2 * TILE, p.v_pages + (size_t)pc.x * kPiece, TILE, bar);
+    }
+    if (pc.y >= 0) {
+      bulk_load(dst + TILE, p.k_pages + (size_t)pc.y * kPiece, TILE, bar);
+      bulk_load(dst + 3 * TILE, p.v_pages + (size_t)pc.y * kPiece, TILE, bar);
+    }
+  };
+  if (producer) {
+    for (int i = 0; i < S && i < n_my; ++i) issue(i);
   }
 
 
