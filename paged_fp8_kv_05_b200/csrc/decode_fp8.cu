@@ -42,8 +42,7 @@
 // ceil(L_b / 32) units of 32 KV tokens for up to RC query rows.  Two modes
 // share all code below the prologue:
 //  * grid: CTA = one split of split_tokens tokens of one segment; the hardware
-//    hands CTAs to SMs as slots free up (split-major order: first splits
-//    first);
+//    hands CTAs to SMs as slots free up;
 //  * balanced: all units of all segments form one list (segments in (b, h, rg)
 //    order) and CTA c of the G CTAs takes units [c*U/G, (c+1)*U/G), so every
 //    CTA streams the same amount of KV whatever the length mix; its range cuts
@@ -287,13 +286,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   // ---- this CTA's range of units and its portions (A1)
   long long u0 = 0, u1 = 0;
   if (p.grid_mode) {
-    // CTA cid is split (cid / segs) of segment (cid % segs): tokens
+    // CTA cid is split (cid % num_splits) of segment (cid / num_splits): tokens
     // [split * T, split * T + T) of it, one portion; a sequence split in n_parts
-    // leaves n_parts partials (slots segment * num_splits + split).  Split-major
-    // order: the first splits, full length for every long sequence, are handed
-    // out first, the shorter or empty last splits fill in behind them.
-    const int n_sg = G / p.num_splits;
-    const int split = cid / n_sg, sg = cid % n_sg;
+    // leaves n_parts partials (slots segment * num_splits + split).  Segment-
+    // major order (the splits of a segment are neighbours) measured 2.5 % faster
+    // than split-major on the LLaMA-shaped and long-context workloads.
+    const int split = cid % p.num_splits, sg = cid / p.num_splits;
     const int b = sg / Hs, seg = sg % Hs;
     const int L = __ldg(p.seq_lens + b);
     if (!valid_len(L)) return;  // CTA-uniform; its rows were zeroed above
