@@ -88,13 +88,17 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The decode kernel and its launch path: the kernel, the shared device helpers
+# and planner, the ABI layer that plans and launches it.
+DECODE_SOURCES = ("atlas_internal.cuh", "atlas_kv.cu", "decode_fp8.cu")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_fp8_kv_05_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -311,6 +315,45 @@ def reference_arm(args):
 
 # ------------------------------------------------------------------ our arm
 
+def append_throughput(w, device, flush_l2, ak, n_new=1024, calls=20):
+    """A0 alone: one atlas_fp8_kv_append of n_new float32 tokens per sequence
+    (the cache-fill shape), into a pool of its own so the workload's cache is
+    untouched.  Bytes per call: 4 (f32 in) + 1 (code out) per element, plus
+    the block-table entries and start positions.  Event-timed per call with
+    the L2 flushed before each; reported beside the step, not in `value`."""
+    B, Hkv, D, ps = w.batch, w.num_kv_heads, w.head_dim, w.page_size
+    pages_per_seq = (n_new + ps - 1) // ps
+    pool = ak.KVPool(B * pages_per_seq, ps, Hkv, D, w.k_scale, w.v_scale, max_batch=B,
+                     max_q_len=1, num_q_heads=Hkv, max_seq_len=n_new, device=device)
+    table = torch.arange(B * pages_per_seq, dtype=torch.int32, device=device).view(B, pages_per_seq)
+    start = torch.zeros(B, dtype=torch.int32, device=device)
+    gen = torch.Generator(device=device).manual_seed(7)
+    k = torch.randn(B, n_new, Hkv, D, device=device, generator=gen)
+    v = torch.randn(B, n_new, Hkv, D, device=device, generator=gen)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(3):
+        ak.atlas_fp8_kv_append(pool, k, v, table, start)
+    times = []
+    for _ in range(calls):
+        flush_l2()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ak.atlas_fp8_kv_append(pool, k, v, table, start)
+        z.record(stream)
+        z.synchronize()
+        times.append(a.elapsed_time(z))
+    if pool.device_error() != 0:
+        raise SystemExit("device error flag set during the append timing")
+    elems = 2 * B * n_new * Hkv * D
+    nbytes = elems * (4 + 1) + 4 * B * pages_per_seq + 4 * B
+    ms = sum(times) / len(times)
+    peak, _ = load_peaks()
+    return {"what": f"atlas_fp8_kv_append, {B} x {n_new} x {Hkv} x {D} float32 K and V",
+            "us_per_call": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / peak, "bytes_per_call": nbytes,
+            "launches_per_call": 1}
+
+
 def ours(args):
     world, rank, local, dist = dist_setup(args)
     if not torch.cuda.is_available():
@@ -404,6 +447,7 @@ def ours(args):
     e2e_total = max_over_ranks(sum(e2e_ms), dist, device)
     if dw.pool.device_error() != 0:
         raise SystemExit("device error flag set during timing")
+    append_line = append_throughput(w, device, flush_l2, ak)
 
     peak, peak_kind = load_peaks()
     step_bytes = b_dec + b_app
@@ -430,6 +474,7 @@ def ours(args):
         "e2e": {"value": world * step_bytes / (e2e_total / K_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "ms_per_step": e2e_total / K_e2e, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "append": append_line,
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }

@@ -15,56 +15,111 @@
 // byte 4*((t%8)/2) + 2*(t/8) + t%2 (bytes 4c..4c+3 hold slots 2c, 2c+1, 2c+8,
 // 2c+9, the token order of the decode kernel's P fragments).
 // Memory-bound: per element 4 (f32) or 2 (bf16) bytes read, 1 byte written.
-// One thread owns 16 consecutive elements of one (sequence, token, head) row:
-// 64 B (or 32 B) of coalesced input, then one 16-byte store into a K page or
-// 16 byte stores (one per head dimension, 16 bytes apart) into a V page.
+// A CTA owns 16 consecutive new tokens of one (sequence, KV head): D/16 x 16
+// threads, each with 16 consecutive elements of one token row of K and of V
+// (64 B or 32 B of coalesced input each).  K codes go out as one 16-byte store
+// per thread.  V codes are transposed through shared memory: when the 16
+// tokens fill one 16-slot group of a page exactly (the cache-fill case), every
+// thread stores whole 16-byte group rows; otherwise (the few tokens of a
+// decode step) each valid code is stored as one byte.  Index arithmetic is
+// 32-bit and done once per CTA.
 #include "atlas_internal.cuh"
 
 namespace atlas {
 namespace {
 
-__global__ void __launch_bounds__(256) fp8_append_kernel(const AppendParams p) {
-  const int chunks = p.D / 16;
-  const long long per_tensor = (long long)p.batch * p.n_new * p.Hkv * chunks;
-  const long long total = 2 * per_tensor;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += stride) {
-    const int which = idx >= per_tensor;   // 0 = K, 1 = V
-    long long r = idx - (which ? per_tensor : 0);
-    const int j = (int)(r % chunks); r /= chunks;
-    const int h = (int)(r % p.Hkv); r /= p.Hkv;
-    const int t = (int)(r % p.n_new);
-    const int b = (int)(r / p.n_new);
+constexpr int kTok = 16;  // tokens per CTA (one 16-slot V group when aligned)
 
-    const int pos = __ldg(p.start_pos + b) + t;
-    const int blk = pos / p.ps;
-    if (pos < 0 || blk >= p.max_blocks) { atomicOr(p.err, ATLAS_DEVERR_APPEND); continue; }
-    const int page = __ldg(p.block_table + (size_t)b * p.max_blocks + blk);
-    if (page < 0 || page >= p.num_pages) { atomicOr(p.err, ATLAS_DEVERR_APPEND); continue; }
+template <int D>
+__global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
+  constexpr int CH = D / 16;  // 16-element chunks per row
+  __shared__ __align__(16) uint8_t s_v[D][kTok];
+  __shared__ int s_page[kTok];
+  const int n_tiles = (p.n_new + kTok - 1) / kTok;
+  const int tile = blockIdx.x % n_tiles;
+  const int bh = blockIdx.x / n_tiles;
+  const int h = bh % p.Hkv, b = bh / p.Hkv;
+  const int t0 = tile * kTok;
+  const int n_tok = min(kTok, p.n_new - t0);
+  const int start = __ldg(p.start_pos + b);
+  const int tid = threadIdx.x;
+  const int lt = tid / CH, j = tid % CH;  // token within the tile, chunk
 
-    const size_t src_elem = ((((size_t)b * p.n_new + t) * p.Hkv + h) * p.D) + 16 * j;
-    float x[16];
-    load16_as_f32(which ? p.v_new : p.k_new, src_elem, p.dtype, x);
-    const uint4 codes = quantize16_e4m3(x, __ldg((which ? p.v_scale : p.k_scale) + h));
+  if (tid < kTok) {  // page of each token of the tile (-1: not written, flagged)
+    int page = -1;
+    const int pos = start + t0 + tid;
+    if (tid < n_tok) {
+      const int blk = pos / p.ps;
+      if (pos >= 0 && blk < p.max_blocks) {
+        page = __ldg(p.block_table + (size_t)b * p.max_blocks + blk);
+        if (page < 0 || page >= p.num_pages) page = -1;
+      }
+      if (page < 0) atomicOr(p.err, ATLAS_DEVERR_APPEND);
+    }
+    s_page[tid] = page;
+  }
+  __syncthreads();
+
+  const int pos = start + t0 + lt;
+  const int page = s_page[lt];
+  if (lt < n_tok && page >= 0) {
+    const size_t src = (((size_t)b * p.n_new + t0 + lt) * p.Hkv + h) * D + 16 * j;
     const size_t head_page = (size_t)page * p.Hkv + h;
-    if (!which)
-      store16_k(p.k_pages, head_page, p.D, p.ps, pos % p.ps, j, codes);
-    else
-      store16_v(p.v_pages, head_page, p.D, p.ps, pos % p.ps, j, codes);
+    float x[16];
+    load16_as_f32(p.k_new, src, p.dtype, x);
+    store16_k(p.k_pages, head_page, D, p.ps, pos % p.ps, j, quantize16_e4m3(x, __ldg(p.k_scale + h)));
+    load16_as_f32(p.v_new, src, p.dtype, x);
+    const uint4 cv = quantize16_e4m3(x, __ldg(p.v_scale + h));
+    const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) s_v[16 * j + k][lt] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
+  }
+  __syncthreads();
+
+  // V: slot t of a 16-slot group sits at byte 4*((t%8)/2) + 2*(t/8) + t%2 of
+  // the group row of each head dimension
+  const int p0 = start + t0;
+  const bool whole_group = n_tok == kTok && (p0 % 16) == 0 && s_page[0] >= 0;
+  if (whole_group) {  // thread d writes row d of the group (16 bytes)
+    const int d = tid;
+    uint32_t word[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) {
+      const int byte = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
+      word[byte >> 2] |= (uint32_t)s_v[d][t] << (8 * (byte & 3));
+    }
+    const size_t head_page = (size_t)s_page[0] * p.Hkv + h;
+    uint8_t* dst = p.v_pages + (head_page * (p.ps / 16) + (p0 % p.ps) / 16) * (16 * D) + 16 * d;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(word[0], word[1], word[2], word[3]);
+  } else {  // byte stores for the valid tokens
+    for (int idx = tid; idx < n_tok * D; idx += D) {
+      const int t = idx / D, d = idx % D;
+      const int pg = s_page[t];
+      if (pg < 0) continue;
+      const int slot = (p0 + t) % p.ps;
+      const int g = slot % 16;
+      const int byte = 4 * ((g & 7) >> 1) + 2 * (g >> 3) + (g & 1);
+      const size_t head_page = (size_t)pg * p.Hkv + h;
+      p.v_pages[(head_page * (p.ps / 16) + slot / 16) * (16 * D) + 16 * d + byte] = s_v[d][t];
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream) {
-  const long long total = 2LL * p.batch * p.n_new * p.Hkv * (p.D / 16);
-  if (total == 0) return cudaSuccess;
-  const int threads = 256;
-  long long blocks = (total + threads - 1) / threads;
-  const long long cap = (long long)num_sms * 8;
-  if (blocks > cap) blocks = cap;
-  fp8_append_kernel<<<(unsigned)blocks, threads, 0, stream>>>(p);
+  (void)num_sms;
+  if (p.batch == 0 || p.n_new == 0) return cudaSuccess;
+  const long long n_tiles = (p.n_new + kTok - 1) / kTok;
+  const long long blocks = n_tiles * p.Hkv * p.batch;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  if (p.D == 128) {
+    fp8_append_kernel<128><<<(unsigned)blocks, 128, 0, stream>>>(p);
+  } else if (p.D == 64) {
+    fp8_append_kernel<64><<<(unsigned)blocks, 64, 0, stream>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
