@@ -49,8 +49,8 @@
  *
  * Threads.  A pool is immutable after creation except for its workspace.
  * Decode calls that share one pool share its workspace, so they must be
- * issued on one stream (or otherwise ordered); appends do not use the
- * workspace.
+ * issued on one stream (or otherwise ordered); appends only set bits of the
+ * workspace's error word.
  */
 #ifndef ATLAS_KV_H
 #define ATLAS_KV_H
@@ -105,9 +105,10 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
  * max_seq_len <= max_seq_len fit with the automatic partition, and -- when
  * min_split_tokens > 0 -- with any split override >= min_split_tokens.
  * The workspace holds the split-KV partial results (float32 O rows and
- * log2-sum-exp values, one slot per segment plus one per CTA), one completion
- * counter per segment (sequence, KV head, row block) and the device error
- * word.  The figure depends on the SM count of the current device (148 if
+ * log2-sum-exp values: one slot per split of every segment with the grid
+ * partition, one per segment plus one per CTA with the balanced one), one
+ * completion counter per segment (sequence, KV head, row block) and the
+ * device error word.  The figure depends on the SM count of the current device (148 if
  * none is visible).  Returns 0 for invalid arguments.
  */
 ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len,
@@ -152,10 +153,11 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
 /* Tuning options for atlas_kv_pool_set_option. */
 #define ATLAS_OPT_SPLIT_TOKENS   1   /* same as atlas_kv_pool_set_split_tokens           */
 #define ATLAS_OPT_STAGES         2   /* K/V staging depth per stream: 0 = auto, 2 or 3   */
-#define ATLAS_OPT_WAVES          3   /* automatic grid: CTAs per resident CTA slot, 0 = 1, */
-                                     /* up to 8 (smaller ranges the hardware schedules    */
-                                     /* as slots free up); the workspace must hold the    */
-                                     /* extra partial slots (ATLAS_ERR_WORKSPACE if not)  */
+#define ATLAS_OPT_WAVES          3   /* automatic sizing, 0 = 1, up to 8: balanced: CTAs */
+                                     /* per resident CTA slot; grid: splits sized for     */
+                                     /* 2 x this many waves of resident CTAs; more, smaller */
+                                     /* parts need more partial slots in the workspace    */
+                                     /* (ATLAS_ERR_WORKSPACE if they do not fit)          */
 #define ATLAS_OPT_PARTITION      4   /* 0 = auto, 1 = grid (CTA = one split of one      */
                                      /* (sequence, KV head, row block); the hardware     */
                                      /* schedules them), 2 = balanced (equal ranges of   */
@@ -201,9 +203,9 @@ ATLAS_API atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const 
  * max_seq_len: host upper bound of seq_lens (bounds the work of one CTA).
  * out: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
  * A sequence with seq_len < q_len, seq_len > max_blocks_per_seq*page_size or
- * seq_len > max_seq_len gets zero output rows and flags ATLAS_DEVERR_SEQ_LEN; a page id outside
- * [0, num_pages) is skipped (its tokens do not take part) and flags
- * ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
+ * seq_len > max_seq_len gets zero output rows and flags ATLAS_DEVERR_SEQ_LEN;
+ * a page id outside [0, num_pages) is skipped (its tokens do not take part)
+ * and flags ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
  * Partition (ATLAS_OPT_PARTITION): each (sequence, KV head, row block)
  * segment is cut into splits of a fixed number of tokens, one CTA each, that
  * the hardware hands to SMs as they free up; or the 32-token units of all
@@ -226,8 +228,8 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, con
  * to atlas_fp8_kv_append(pool, k_new, v_new, dtype, block_table,
  * max_blocks_per_seq, start_pos = seq_lens - q_len, batch, q_len) followed by
  * atlas_paged_gqa_decode on the pool's pages and scales: the pages end up
- * bit-identical and so does the output.  Every CTA whose range holds a new
- * token quantises and writes it, then reads it back with the rest of its range.
+ * bit-identical and so does the output.  Every CTA whose split (or range)
+ * holds a new token quantises and writes it, then reads it back with the rest.
  * k_new / v_new: device [batch][q_len][num_kv_heads][head_dim] of dtype, 16-byte
  * aligned.  A new token whose page id is outside [0, num_pages) is not written
  * and flags ATLAS_DEVERR_APPEND (and ATLAS_DEVERR_PAGE_ID for the decode).
