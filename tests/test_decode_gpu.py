@@ -83,6 +83,9 @@ EDGE = [
     (2, 12, 4, 64, 32, [95, 97], 3),             # page 32, D 64, G 3, q_len 3
     (1, 8, 1, 128, 16, [1000], 2),
     (5, 8, 2, 128, 48, [47, 48, 49, 96, 1], 1),  # page 48
+    (2, 8, 2, 128, 1024, [1500, 3000], 1),       # largest page size
+    (2, 40, 8, 64, 16, [300, 77], 5),            # D 64, two warps per K/V stream
+    (2, 64, 1, 64, 16, [500, 33], 1),            # D 64, four warps per stream (balanced)
 ]
 
 
