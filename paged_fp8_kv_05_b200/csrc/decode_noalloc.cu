@@ -15,7 +15,7 @@
 // contents; each call clears the counters and the error word (the only parts
 // that must start at zero) with cudaMemsetAsync on its stream before the
 // launch.  Calls whose kernels overlap on the GPU (different streams, no
-// ordering) race on the array.  If the split-KV partials of the balanced
+// ordering) race on the array.  If the split-KV partials of the automatic
 // partition would not fit, the call runs one CTA per (sequence, KV head, row
 // group) segment, which writes no partials; a call that would then need a
 // segment longer than 65536 tokens is rejected with ATLAS_ERR_WORKSPACE.
