@@ -167,6 +167,17 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
                                      /* of 4, 8, 16, 32, 64 holding q_len * G), else one */
                                      /* of those; fewer rows make more row blocks, each  */
                                      /* streaming the KV head's pages again              */
+#define ATLAS_OPT_WAIT_LIMIT_US  6   /* wall-clock limit of every bounded wait inside the */
+                                     /* decode kernel, in microseconds: 0 = the default  */
+                                     /* (200 ms), else 1 .. 10^7                          */
+#define ATLAS_OPT_TEST_SKIP_UNIT 7   /* TESTS ONLY: -1 = off (default); k >= 0 = the     */
+                                     /* first K/V stream of CTA 0 never issues the copies */
+                                     /* of its k-th unit, so the wait for them runs out: */
+                                     /* the call flags ATLAS_DEVERR_TIMEOUT, the output   */
+                                     /* rows of the affected (sequence, KV head) are      */
+                                     /* unspecified, every other one is computed, and no  */
+                                     /* copy is left in flight.  Exercises the bounded-   */
+                                     /* wait error path without any fault                 */
 
 /*
  * Set a tuning option of later decode calls (see ATLAS_OPT_*).  Values out of

@@ -32,6 +32,8 @@ OPT_STAGES = 2
 OPT_WAVES = 3
 OPT_PARTITION = 4
 OPT_ROWS_PER_CTA = 5
+OPT_WAIT_LIMIT_US = 6
+OPT_TEST_SKIP_UNIT = 7
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 

@@ -55,7 +55,15 @@ struct DecodeParams {
   const void* k_new;          // [B][q_len][Hkv][D] f32 or bf16, or nullptr
   const void* v_new;
   int new_dtype;              // ATLAS_DTYPE_*
+  // bounded waits: wall-clock limit of every mbarrier wait (ns)
+  unsigned long long wait_limit_ns;
+  // test-only lost-copy injection: when >= 0, CTA 0's first K/V stream never
+  // issues the bulk copies of its unit number test_skip_unit, so the wait for
+  // them runs out (no copy is in flight for that stage); -1 in normal use
+  int test_skip_unit;
 };
+
+constexpr unsigned long long kDefaultWaitLimitNs = 200ull * 1000 * 1000;
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
 

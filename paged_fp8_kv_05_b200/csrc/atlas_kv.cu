@@ -22,6 +22,8 @@ struct atlas_kv_pool {
   int32_t waves_override;
   int32_t partition_override;
   int32_t rows_override;
+  int32_t wait_limit_us;   // 0: the default limit of every bounded wait
+  int32_t test_skip_unit;  // -1: normal; >= 0: lost-copy injection (tests only)
   size_t counters_bytes;  // largest counter block any accepted call uses
 };
 
@@ -189,6 +191,8 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   p->waves_override = 0;
   p->partition_override = 0;
   p->rows_override = 0;
+  p->wait_limit_us = 0;
+  p->test_skip_unit = -1;
   p->counters_bytes = counters_bytes;
   *out = p;
   return ATLAS_OK;
@@ -229,6 +233,14 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
       if (value != 0 && value != 4 && value != 8 && value != 16 && value != 32 && value != 64)
         return ATLAS_ERR_INVALID_ARG;
       pool->rows_override = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_WAIT_LIMIT_US:
+      if (value < 0 || value > 10 * 1000 * 1000) return ATLAS_ERR_INVALID_ARG;
+      pool->wait_limit_us = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_TEST_SKIP_UNIT:
+      if (value < -1) return ATLAS_ERR_INVALID_ARG;
+      pool->test_skip_unit = value;
       return ATLAS_OK;
   }
   return ATLAS_ERR_INVALID_ARG;
@@ -363,6 +375,9 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.k_new = k_new;
   p.v_new = v_new;
   p.new_dtype = new_dtype;
+  p.wait_limit_ns = pool->wait_limit_us > 0 ? 1000ull * pool->wait_limit_us
+                                            : atlas::kDefaultWaitLimitNs;
+  p.test_skip_unit = pool->test_skip_unit;
   cudaError_t e = atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid,
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;

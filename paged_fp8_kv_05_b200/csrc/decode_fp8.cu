@@ -60,9 +60,9 @@
 // CTA is written out as bf16, otherwise the CTA writes (O/l, log2-sum-exp) to
 // its part's slot and the CTA that finishes the segment last -- one atomic
 // counter per segment, no waiting -- merges the parts and resets the counter.
-// Every mbarrier wait is bounded (200 ms of wall clock): a wait that runs out
-// flags ATLAS_DEVERR_TIMEOUT and the warp stops computing after draining its
-// loads.
+// Every mbarrier wait is bounded (p.wait_limit_ns of wall clock, 200 ms by
+// default): a wait that runs out flags ATLAS_DEVERR_TIMEOUT and the warp stops
+// computing after draining its loads.
 #include <float.h>
 #include <math.h>
 
@@ -74,7 +74,6 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
 constexpr int kUnit = 32;  // tokens per pipeline unit (two 16-token pieces)
 constexpr int kQBuf = 3;   // Q row buffers: portion pi + 2 loads while pi computes
 
@@ -497,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const int st = i % S;
     uint64_t* bar = &full_bar[stream * S + st];
     uint8_t* dst = ring + (size_t)(stream * S + st) * STAGE;
+    if (p.test_skip_unit == i && cid == 0 && stream == 0) return;  // lost copy (tests only)
     const int2 pc = s_pieces[stream + NSTREAM * i];
     const uint32_t bytes = (pc.x >= 0 ? 2 * TILE : 0) + (pc.y >= 0 ? 2 * TILE : 0);
     if (bytes == 0) {
@@ -833,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       if (k >= ke) break;
       const int st = i_next % S;
       const uint32_t par = (uint32_t)((i_next / S) & 1);
-      if (!mbar_wait_bounded(&full_bar[stream * S + st], par, kWaitLimitNs)) {
+      if (!mbar_wait_bounded(&full_bar[stream * S + st], par, p.wait_limit_ns)) {
         aborted = true;
         break;
       }
@@ -850,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       }
       if (producer && i_next + S < n_my) {
         if constexpr (RBG > 1) {
-          if (!mbar_wait_bounded(&empty_bar[stream * S + st], par, kWaitLimitNs)) aborted = true;
+          if (!mbar_wait_bounded(&empty_bar[stream * S + st], par, p.wait_limit_ns)) aborted = true;
         }
         // the stage's readers are done: RBG = 1, their loads fed this warp's MMAs
         // before the __syncwarp; RBG > 1, the empty barrier ordered them
@@ -977,7 +977,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     if (lane == 0) atomicOr(p.err, ATLAS_DEVERR_TIMEOUT);
     // drain this stream's loads still in flight (issued: i < min(n_my, i_next + S))
     for (int i = i_next; i < n_my && i < i_next + S; ++i)
-      mbar_wait_bounded(&full_bar[stream * S + i % S], (uint32_t)((i / S) & 1), kWaitLimitNs);
+      mbar_wait_bounded(&full_bar[stream * S + i % S], (uint32_t)((i / S) & 1), p.wait_limit_ns);
     cp_async_wait_all();
     return;
   }

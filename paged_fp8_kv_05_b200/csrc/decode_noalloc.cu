@@ -35,6 +35,12 @@ namespace {
 constexpr size_t kScratchBytes = 8u << 20;  // 8 MiB per GPU
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
+// Longest segment the one-CTA-per-segment fallback accepts.  Its CTA keeps a
+// table of the segment's 32-token units in shared memory: 65536 tokens make
+// 2048 entries of 8 bytes (16 KB), well inside the kernel's shared-memory
+// budget.  (atlas::kMaxUnitsPerCta bounds the ranges of the balanced
+// partition, which this fallback does not use.)
+constexpr int kMaxWholeSegmentTokens = 65536;
 
 __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
 
@@ -101,7 +107,7 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   if (o_off + rows * head_dim * sizeof(float) > kScratchBytes) {
     const int whole = (int)(((long long)max_seq_len + 63) / 64 * 64);
     // one segment's unit table lives in shared memory: bound its length
-    if (whole > 64 * atlas::kMaxUnitsPerCta) return ATLAS_ERR_WORKSPACE;
+    if (whole > kMaxWholeSegmentTokens) return ATLAS_ERR_WORKSPACE;
     L = atlas::plan_decode(batch, num_q_heads, num_kv_heads, q_len, max_seq_len, sms, whole, 0,
                            atlas::kPartitionGrid);
     lse_off = o_off = counters_off;
@@ -147,6 +153,8 @@ extern "C" atlas_status_t atlas_paged_gqa_decode_noalloc(
   p.qk_scale_log2 = (float)(scale * 1.4426950408889634);  // log2(e)
   p.k_new = nullptr;  // decode only
   p.v_new = nullptr;
+  p.wait_limit_ns = atlas::kDefaultWaitLimitNs;
+  p.test_skip_unit = -1;
   cudaError_t e = atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid, s);
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

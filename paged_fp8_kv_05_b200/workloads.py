@@ -6,7 +6,7 @@ CPU oracle take their inputs from here, so the two see identical values.
 
 Recipe (all draws from ``numpy.random.default_rng`` on children of
 ``numpy.random.SeedSequence(seed)``; one child per purpose, in this order:
-lengths, page table, q, k, v, outlier rows, fragmentation):
+lengths, page table, q, k, v, outlier rows, fragmentation, sharp shaping):
 
 * context lengths ``L_b`` per the workload (uniform integers, or
   ``floor(exp(U[ln lo, ln hi]))`` for the log-uniform mix);
@@ -14,6 +14,12 @@ lengths, page table, q, k, v, outlier rows, fragmentation):
 * K and V ``N(0, 1)`` float32 ``[sum L_b, Hkv, D]``; optionally a Bernoulli
   fraction of K rows (one row = one token of one KV head) multiplied by a
   factor *before* the scales are taken (outlier keys);
+* optional sharp-attention shaping of the same draws, before the scales are
+  taken: Q multiplied by a gain (score standard deviation = gain); "needle"
+  keys, a K row replaced by a multiple of one query row of its group, at
+  seeded positions (one inside the MTP drafts when q_len > 1); or a "ramp", K
+  rows of one query head per KV head set to ``c_t * q`` so that its scores
+  rise linearly along the context;
 * per-KV-head scales ``amax_h / 448`` in float32, the amax over every token of
   the generated tensor (new tokens included): one static scale per KV head and
   tensor;
@@ -168,12 +174,53 @@ def _table_frag(rng, lengths, page_size, num_pages, length_spec, rounds=8, per_r
     return table
 
 
+def _shape_scores(rng, q, k, L, cu, num_kv_heads, q_len, needles, needle_gain, ramp):
+    """Sharp-attention shaping of the K draws (in place).  Pure input layout:
+    K rows become multiples of query rows, chosen by the seeded ``rng``.
+
+    * ``needles`` per sequence and KV head: position t (uniform over the
+      context; the first one inside the last q_len positions when q_len > 1),
+      a q-head of the group and a query row that sees t; the K row becomes
+      ``needle_gain * q`` of that row.
+    * ``ramp`` > 0: for every sequence and KV head, the K rows become
+      ``(ramp * t * sqrt(D) / |q|^2) * q`` for q the last query row of the
+      group's first q-head, so that this row's score ``q . k_t / sqrt(D)`` is
+      ``ramp * t`` (before FP8 rounding): it rises along the whole context.
+    """
+    B = len(L)
+    Hq, D = q.shape[2], q.shape[3]
+    G = Hq // num_kv_heads
+    for b in range(B):
+        n = int(L[b])
+        base = int(cu[b])
+        for h in range(num_kv_heads):
+            for j in range(needles):
+                if j == 0 and q_len > 1:
+                    t = int(rng.integers(n - q_len, n))
+                else:
+                    t = int(rng.integers(0, n))
+                i_min = max(0, t - (n - q_len))
+                i = int(rng.integers(i_min, q_len))
+                hq = h * G + int(rng.integers(0, G))
+                k[base + t, h, :] = np.float32(needle_gain) * q[b, i, hq, :]
+            if ramp > 0:
+                qr = q[b, q_len - 1, h * G, :].astype(np.float64)
+                nq = float(qr @ qr)
+                if nq > 0:
+                    c = ramp * np.arange(n, dtype=np.float64) * np.sqrt(D) / nq
+                    k[base:base + n, h, :] = (c[:, None] * qr[None, :]).astype(np.float32)
+
+
 def make_workload(*, batch, num_q_heads, num_kv_heads, head_dim, page_size, q_len,
                   num_pages, lengths, table="perm", outlier_frac=0.0,
-                  outlier_gain=8.0, seed=0, name="custom") -> Workload:
+                  outlier_gain=8.0, seed=0, name="custom", q_gain=1.0, needles=0,
+                  needle_gain=1.0, ramp=0.0) -> Workload:
     """Draw one workload.  ``lengths`` is ``("fixed", [..])``,
-    ``("uniform", lo, hi)`` (inclusive) or ``("loguniform", lo, hi)``."""
-    (s_len, s_tab, s_q, s_k, s_v, s_out, s_frag) = np.random.SeedSequence(seed).spawn(7)
+    ``("uniform", lo, hi)`` (inclusive) or ``("loguniform", lo, hi)``.
+    ``q_gain``, ``needles``/``needle_gain`` and ``ramp`` shape the draws for
+    sharp attention (see :func:`_shape_scores`)."""
+    (s_len, s_tab, s_q, s_k, s_v, s_out, s_frag,
+     s_sharp) = np.random.SeedSequence(seed).spawn(8)
     L = _lengths(np.random.default_rng(s_len), lengths, batch)
     assert len(L) == batch
     if table == "perm":
@@ -185,6 +232,8 @@ def make_workload(*, batch, num_q_heads, num_kv_heads, head_dim, page_size, q_le
 
     qf = np.random.default_rng(s_q).standard_normal(
         (batch, q_len, num_q_heads, head_dim), dtype=np.float32)
+    if q_gain != 1.0:
+        qf *= np.float32(q_gain)
     q = torch.from_numpy(qf).to(torch.bfloat16)
 
     total = int(L.sum())
@@ -192,6 +241,12 @@ def make_workload(*, batch, num_q_heads, num_kv_heads, head_dim, page_size, q_le
                                                    dtype=np.float32)
     v = np.random.default_rng(s_v).standard_normal((total, num_kv_heads, head_dim),
                                                    dtype=np.float32)
+    cu = np.zeros(batch + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(L)
+    if (needles > 0 or ramp > 0) and total:
+        qv = q.float().numpy()     # the exact bf16 values
+        _shape_scores(np.random.default_rng(s_sharp), qv, k, L, cu, num_kv_heads, q_len,
+                      needles, needle_gain, ramp)
     n_out = 0
     if outlier_frac > 0 and total:
         rows = np.random.default_rng(s_out).random((total, num_kv_heads)) < outlier_frac
@@ -205,14 +260,13 @@ def make_workload(*, batch, num_q_heads, num_kv_heads, head_dim, page_size, q_le
         amax = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
         return (amax / np.float32(FP8_MAX)).astype(np.float32)
 
-    cu = np.zeros(batch + 1, dtype=np.int64)
-    cu[1:] = np.cumsum(L)
     return Workload(name=name, batch=batch, num_q_heads=num_q_heads,
                     num_kv_heads=num_kv_heads, head_dim=head_dim, page_size=page_size,
                     q_len=q_len, num_pages=num_pages, seq_lens=L.astype(np.int32),
                     block_table=bt, q=q, k=k, v=v, k_scale=scale_of(k),
                     v_scale=scale_of(v), cu_seqlens=cu,
-                    meta=dict(seed=seed, outlier_rows=n_out, table=table))
+                    meta=dict(seed=seed, outlier_rows=n_out, table=table, q_gain=q_gain,
+                              needles=needles, needle_gain=needle_gain, ramp=ramp))
 
 
 def config_workload(index: int, seed: int = 0) -> Workload:

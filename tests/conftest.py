@@ -26,3 +26,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    # measured error of every parity check that ran (GPU runs): case, max-abs, rel-L2
+    try:
+        from parity import PARITY_LOG
+    except Exception:
+        return
+    if not PARITY_LOG:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "parity against the float64 oracle (bound: max-abs 1e-2, rel-L2 5e-3)")
+    for case, max_abs, rel in PARITY_LOG:
+        tr.write_line(f"{case:<72s} max-abs {max_abs:.3e}  rel-L2 {rel:.3e}")

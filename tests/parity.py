@@ -76,6 +76,15 @@ def errors(got, ref):
     return max_abs, rel
 
 
+# (case, max-abs, rel-L2) of every parity check of the run, printed at the end
+# of the session by tests/conftest.py
+PARITY_LOG = []
+
+
+def record_parity(case, max_abs, rel):
+    PARITY_LOG.append((case, float(max_abs), float(rel)))
+
+
 def assert_close(got, ref, what=""):
     max_abs, rel = errors(got, ref)
     assert np.all(np.isfinite(np.asarray(got, np.float64)[np.isfinite(ref)])), f"{what}: non-finite output"
@@ -83,5 +92,5 @@ def assert_close(got, ref, what=""):
     return max_abs, rel
 
 
-__all__ = ["oracle_pages", "oracle_decode", "errors", "assert_close", "MAX_ABS", "REL_L2",
-           "paged"]
+__all__ = ["oracle_pages", "oracle_decode", "errors", "assert_close", "record_parity",
+           "PARITY_LOG", "MAX_ABS", "REL_L2", "paged"]

@@ -135,7 +135,11 @@ def test_pool_create_ok_and_plan_is_host_only():
         for bad in (-64, 32, 100, 16384):
             assert ak._lib.atlas_kv_pool_set_split_tokens(h, bad) == ak.ATLAS_ERR_INVALID_ARG
         for opt, val, st in ((ak.OPT_STAGES, 3, 0), (ak.OPT_STAGES, 2, 0), (ak.OPT_STAGES, 0, 0),
-                             (ak.OPT_STAGES, 4, -1), (ak.OPT_SPLIT_TOKENS, 256, 0), (99, 1, -1)):
+                             (ak.OPT_STAGES, 4, -1), (ak.OPT_SPLIT_TOKENS, 256, 0), (99, 1, -1),
+                             (ak.OPT_WAIT_LIMIT_US, 1000, 0), (ak.OPT_WAIT_LIMIT_US, 0, 0),
+                             (ak.OPT_WAIT_LIMIT_US, -1, -1), (ak.OPT_WAIT_LIMIT_US, 10**8, -1),
+                             (ak.OPT_TEST_SKIP_UNIT, 3, 0), (ak.OPT_TEST_SKIP_UNIT, -1, 0),
+                             (ak.OPT_TEST_SKIP_UNIT, -2, -1)):
             assert ak._lib.atlas_kv_pool_set_option(h, opt, val) == st
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 5, 8, 1, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG
         assert ak._lib.atlas_paged_gqa_decode_plan(h, 2, 8, 6, 100, buf, 7) == ak.ATLAS_ERR_INVALID_ARG

@@ -10,7 +10,7 @@ from oracle import attention
 from oracle.paged import GROUP_POS
 from paged_fp8_kv_05_b200 import build, workloads
 
-from parity import assert_close, errors, oracle_decode, oracle_pages
+from parity import assert_close, errors, oracle_decode, oracle_pages, record_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -47,21 +47,27 @@ def test_named_workload_full_output(ak, cfg, partition):
     assert dw.pool.device_error() == 0
     ref = _oracle_named(cfg, w)
     max_abs, rel = assert_close(got, ref, f"config {cfg}, partition {partition}")
+    record_parity(f"config {cfg}, partition {partition}", max_abs, rel)
     print(f"config {cfg}: max-abs {max_abs:.3e} rel-L2 {rel:.3e} plan {dw.plan()}")
 
 
-def test_long_context_sampled_sequences(ak):
+def test_long_context_every_sequence(ak):
+    """The long-context workload (B=4, 65k-131k tokens, 1 % of key rows x8
+    before quantisation): every output element of all four sequences against
+    the oracle, with the automatic plan (several splits per sequence)."""
     w = workloads.config_workload(3)
     dw = _dw(w)
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
     plan = dw.plan()
     assert plan["num_splits"] > 1
-    sample = [0, 2]
-    ref = oracle_decode(w, sequences=sample)
-    max_abs, rel = assert_close(got[sample], ref[sample], "config 3 (sequences 0, 2)")
+    del dw
+    torch.cuda.empty_cache()
+    ref = oracle_decode(w)
+    assert np.all(np.isfinite(ref))
+    max_abs, rel = assert_close(got, ref, "config 3 (all sequences)")
+    record_parity("config 3, all 4 sequences", max_abs, rel)
     print(f"config 3: max-abs {max_abs:.3e} rel-L2 {rel:.3e} plan {plan}")
-    assert np.all(np.isfinite(got))
 
 
 def _case(B, Hq, Hkv, D, ps, lens, q_len, seed=0, P=None, table="perm"):
@@ -238,6 +244,36 @@ def test_bad_inputs_flag_device_errors_without_faulting(ak):
     # the library stays usable
     dw.decode()
     assert dw.pool.device_error() == 0
+
+
+def test_lost_copy_times_out_and_the_library_stays_usable(ak):
+    """Bounded-wait error path, without any fault: CTA 0's first K/V stream
+    never issues the bulk copies of its second unit (a test-only pool option),
+    so nothing is ever in flight for that stage and the wait for it runs out
+    after 1 ms.  The call must flag ATLAS_DEVERR_TIMEOUT and return; every
+    (sequence, KV head) other than CTA 0's -- sequence 0, KV head 0 in the grid
+    partition -- must still match the oracle, and the next normal call on the
+    same pool must be clean and match everywhere."""
+    w = _case(4, 32, 8, 128, 16, [700, 1500, 64, 300], 1, seed=12)
+    dw = _dw(w)
+    dw.pool.set_option(ak.OPT_PARTITION, 1)
+    dw.pool.set_option(ak.OPT_WAIT_LIMIT_US, 1000)
+    dw.pool.set_option(ak.OPT_TEST_SKIP_UNIT, 1)
+    out = torch.full_like(dw.q, float("nan"))
+    dw.decode(out=out)
+    err = dw.pool.device_error()
+    assert err & ak.DEVERR_TIMEOUT, err
+    ref = oracle_decode(w)
+    got = out.float().cpu().numpy()
+    G = w.num_q_heads // w.num_kv_heads
+    keep = np.ones(got.shape[:3], bool)
+    keep[0, :, 0:G] = False                         # sequence 0, KV head 0: unspecified
+    assert_close(got[keep], ref[keep], "segments other than the timed-out one")
+    dw.pool.set_option(ak.OPT_TEST_SKIP_UNIT, -1)
+    dw.pool.set_option(ak.OPT_WAIT_LIMIT_US, 0)
+    again = dw.decode(out=torch.empty_like(dw.q))
+    assert dw.pool.device_error() == 0
+    assert_close(again.float().cpu().numpy(), ref, "the call after the timeout")
 
 
 def test_empty_batch_is_a_noop(ak):
