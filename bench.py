@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--waves", type=int, default=0, help="CTAs per resident CTA slot")
     ap.add_argument("--partition", type=int, default=0, help="0 auto, 1 grid, 2 balanced")
     ap.add_argument("--rows-per-cta", type=int, default=0, help="query rows per CTA (0 auto)")
+    ap.add_argument("--kernel", type=int, default=0,
+                    help="0 auto, 1 FP8 warp-MMA kernel, 2 tensor-core (tcgen05) kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -99,7 +101,7 @@ def load_peaks():
 
 # The decode kernel and its launch path: the kernel, the shared device helpers
 # and planner, the ABI layer that plans and launches it.
-DECODE_SOURCES = ("atlas_internal.cuh", "atlas_kv.cu", "decode_fp8.cu")
+DECODE_SOURCES = ("atlas_internal.cuh", "atlas_kv.cu", "decode_fp8.cu", "decode_tc.cu")
 
 
 def kernel_source_hash():
@@ -369,6 +371,42 @@ def append_throughput(w, device, flush_l2, ak, n_new=1024, calls=20):
             "launches_per_call": 1}
 
 
+def accept_throughput(device, flush_l2, ak, batch=128, num_drafts=4, vocab=151936, calls=20):
+    """Greedy MTP acceptance alone (the step after a verify decode): bf16
+    verify logits [batch, K + 1, vocab] read once, plus the drafts in and the
+    targets, accepted counts and next tokens out.  Event-timed per call with
+    the L2 flushed before each; reported beside the decode step."""
+    from paged_fp8_kv_05_b200 import workloads
+    logits, drafts, _ = workloads.make_verify_logits(batch=batch, num_drafts=num_drafts,
+                                                     vocab=vocab, seed=3)
+    lg = logits.to(device).contiguous()
+    dr = torch.from_numpy(drafts).to(device).contiguous()
+    pool = ak.KVPool(4, 16, 1, 64, [1.0], [1.0], max_batch=batch, max_q_len=1, num_q_heads=1,
+                     max_seq_len=16, device=device)
+    n, nxt, tg = ak.atlas_mtp_greedy_accept(pool, lg, dr)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(3):
+        ak.atlas_mtp_greedy_accept(pool, lg, dr, targets=tg, n_accepted=n, next_token=nxt)
+    times = []
+    for _ in range(calls):
+        flush_l2()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ak.atlas_mtp_greedy_accept(pool, lg, dr, targets=tg, n_accepted=n, next_token=nxt)
+        z.record(stream)
+        z.synchronize()
+        times.append(a.elapsed_time(z))
+    if pool.device_error() != 0:
+        raise SystemExit("device error flag set during the acceptance timing")
+    nbytes = lg.numel() * lg.element_size() + dr.numel() * 4 + tg.numel() * 4 + 2 * batch * 4
+    ms = sum(times) / len(times)
+    peak, _ = load_peaks()
+    return {"what": f"atlas_mtp_greedy_accept, bf16 logits {batch} x {num_drafts + 1} x {vocab}",
+            "us_per_call": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / peak, "bytes_per_call": nbytes,
+            "launches_per_call": 1}
+
+
 def measure(index, args, device, dist, ak, flush_l2, local):
     """Time K fused steps (append + decode, one launch each) of one workload,
     then K_e2e steps end to end through the public API with pinned host
@@ -388,6 +426,8 @@ def measure(index, args, device, dist, ak, flush_l2, local):
         dw.pool.set_option(ak.OPT_PARTITION, args.partition)
     if args.rows_per_cta:
         dw.pool.set_option(ak.OPT_ROWS_PER_CTA, args.rows_per_cta)
+    if args.kernel:
+        dw.pool.set_option(ak.OPT_KERNEL, args.kernel)
     plan = dw.plan()
     b_dec, b_app = algorithmic_bytes(w)
     stream = torch.cuda.current_stream(device)
@@ -467,8 +507,10 @@ def measure(index, args, device, dist, ak, flush_l2, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / 8000.0,
-                     "kernel": "paged_decode_fp8_kernel (fused append + decode, one launch "
-                               "per step, launch-averaged over the timed steps)",
+                     "kernel": ("paged_decode_tc_kernel" if plan["kernel"] == 3 else
+                                "paged_decode_fp8_kernel") +
+                               " (fused append + decode, one launch per step, launch-averaged "
+                               "over the timed steps)",
                      "traffic": recorded_traffic(index),
                      "algorithmic_bytes": step_bytes,
                      "algorithmic_flops": algorithmic_flops(w)},
@@ -529,6 +571,7 @@ def ours(args):
         "clocks": h["clocks"],
         "per_config": per,
         "append": append_line,
+        "accept": accept_throughput(device, flush_l2, ak),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(head_w, args.cpu_seconds)

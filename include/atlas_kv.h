@@ -14,9 +14,14 @@
  * rounding or mask convention; the readings used here are:
  *
  *   pages        uint8 E4M3 codes; K pages token-major
- *                [num_pages][num_kv_heads][page_size][head_dim]; V pages in
- *                16-slot groups, head-dim-major inside a group:
- *                [num_pages][num_kv_heads][page_size/16][head_dim][16]
+ *                [num_pages][num_kv_heads][page_size][head_dim], and with
+ *                head_dim 128 each 128-byte token row stores its 16-byte
+ *                chunk j (dims 16j..16j+15) at chunk position j XOR (slot % 8)
+ *                (the tensor cores' 128-byte swizzle, so pages are copied
+ *                into shared memory verbatim); V pages in 16-slot groups,
+ *                head-dim-major inside a group:
+ *                [num_pages][num_kv_heads][page_size/16][head_dim][16], slot t
+ *                of a group at byte 4*((t%8)/2) + 2*(t/8) + t%2
  *   block table  int32 [batch][max_blocks_per_seq]; token p of sequence b is in
  *                page block_table[b][p / page_size], slot p % page_size
  *   scales       one float32 per KV head for K and one for V (static)
@@ -91,8 +96,10 @@ typedef enum { ATLAS_DTYPE_F32 = 0, ATLAS_DTYPE_BF16 = 1 } atlas_dtype_t;
 #define ATLAS_PLAN_SPLIT_TOKENS  0   /* KV tokens per split / per CTA range           */
 #define ATLAS_PLAN_NUM_SPLITS    1   /* splits (grid) or most ranges (balanced) of a  */
                                      /* max-length segment                            */
-#define ATLAS_PLAN_KERNEL        2   /* FP8 mma.sync kernel (E4M3 tensor cores) with  */
-                                     /* 1 = grid partition, 2 = balanced partition    */
+#define ATLAS_PLAN_KERNEL        2   /* 1 = FP8 warp-MMA kernel (mma.sync E4M3), grid */
+                                     /* partition; 2 = the same, balanced partition;  */
+                                     /* 3 = 5th-generation tensor-core kernel         */
+                                     /* (tcgen05.mma, TMEM accumulators), grid        */
 #define ATLAS_PLAN_ROWS_PER_CTA  3   /* query rows (q_len x group) per segment        */
 #define ATLAS_PLAN_ROW_BLOCKS    4   /* segments per (sequence, KV head)              */
 #define ATLAS_PLAN_LAUNCHES      5   /* kernel launches per decode call               */
@@ -119,7 +126,8 @@ ATLAS_API size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len,
 /*
  * Describe a page pool.  num_pages >= 1; page_size a multiple of 16 and
  * <= 1024; head_dim 64 or 128; num_kv_heads >= 1.  k_pages: device uint8
- * [num_pages][num_kv_heads][page_size][head_dim] (token-major); v_pages:
+ * [num_pages][num_kv_heads][page_size][head_dim] (token-major; chunk-permuted
+ * rows when head_dim is 128, see the page layout above); v_pages:
  * device uint8 [num_pages][num_kv_heads][page_size/16][head_dim][16] (16-slot
  * groups, head-dim-major inside a group); both 16-byte aligned.
  * k_scale / v_scale: device float32 [num_kv_heads] (used by append; decode
@@ -167,12 +175,21 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
                                      /* of 4, 8, 16, 32, 64 holding q_len * G), else one */
                                      /* of those; fewer rows make more row blocks, each  */
                                      /* streaming the KV head's pages again              */
+#define ATLAS_OPT_KERNEL         8   /* 0 = auto (the tensor-core kernel when head_dim  */
+                                     /* is 128 and q_len * G >= 16, where QK^T and PV   */
+                                     /* are real contractions), 1 = FP8 warp-MMA kernel, */
+                                     /* 2 = tensor-core kernel (head_dim 128 only, else  */
+                                     /* ATLAS_ERR_UNSUPPORTED); the tensor-core kernel   */
+                                     /* runs blocks of 64 query rows in the grid         */
+                                     /* partition (ATLAS_OPT_PARTITION and              */
+                                     /* ATLAS_OPT_ROWS_PER_CTA do not apply to it)      */
 #define ATLAS_OPT_WAIT_LIMIT_US  6   /* wall-clock limit of every bounded wait inside the */
                                      /* decode kernel, in microseconds: 0 = the default  */
                                      /* (200 ms), else 1 .. 10^7                          */
 #define ATLAS_OPT_TEST_SKIP_UNIT 7   /* TESTS ONLY: -1 = off (default); k >= 0 = the     */
                                      /* first K/V stream of CTA 0 never issues the copies */
-                                     /* of its k-th unit, so the wait for them runs out: */
+                                     /* of its k-th unit (tensor-core kernel: of its k-th */
+                                     /* 128-token tile), so the wait for them runs out:  */
                                      /* the call flags ATLAS_DEVERR_TIMEOUT, the output   */
                                      /* rows of the affected (sequence, KV head) are      */
                                      /* unspecified, every other one is computed, and no  */
@@ -289,6 +306,30 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode_noalloc(
 ATLAS_API atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t batch,
                                            int32_t num_q_heads, int32_t q_len,
                                            int32_t max_seq_len, int32_t* plan, int32_t n);
+
+/*
+ * Greedy acceptance of MTP draft tokens, the step after an MTP-verify decode
+ * (GB10 page: MTP with K = 4 drafts; the speculative-decoding page,
+ * blog.hotdry.top: draft -> verify -> accept).  logits: device
+ * [batch][num_drafts + 1][vocab] of dtype (float32 or bf16), finite values;
+ * row i scores the token after new position i of the verify step.  drafts:
+ * device int32 [batch][num_drafts].  Writes, for every sequence:
+ *   targets    device int32 [batch][num_drafts + 1]: first argmax of each row
+ *              (ties to the lowest token id)
+ *   n_accepted device int32 [batch]: leading drafts equal to their target
+ *   next_token device int32 [batch]: targets[b][n_accepted[b]], the token
+ *              emitted after the accepted drafts
+ * One kernel; each logits row is read once.  Uses batch completion counters
+ * of the pool's workspace (zero before and after; issue on the stream of the
+ * pool's decode calls).  batch <= the pool's max_batch; batch == 0 is a
+ * no-op.  Exact: integer results equal the definition bit for bit.
+ */
+ATLAS_API atlas_status_t atlas_mtp_greedy_accept(const atlas_kv_pool_t* pool, const void* logits,
+                                                 int32_t dtype, int32_t batch,
+                                                 int32_t num_drafts, int32_t vocab,
+                                                 const int32_t* drafts, int32_t* targets,
+                                                 int32_t* n_accepted, int32_t* next_token,
+                                                 void* stream);
 
 /*
  * Wait for the stream, read the pool's device error word into *code and

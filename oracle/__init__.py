@@ -25,9 +25,16 @@ What it computes, and where the sources say so:
   "Attention" paragraph: dedicated MQA/GQA kernels; GB10 page: MTP with
   K = 4 drafts).
 
+* ``acceptance`` -- greedy acceptance of MTP draft tokens: the target's
+  choice at each new position is the first maximum of the verify logits;
+  leading drafts equal to it are accepted, and the target at the first
+  position not covered is emitted (GB10 page: MTP with K = 4; the
+  speculative-decoding fusion page, blog.hotdry.top: the draft -> verify ->
+  accept loop).
+
 Every function is pinned by ``tests/test_oracle_*.py`` against something
 other than itself (closed forms, brute force, invariants, torch's own
 float8 and SDPA routines).  No function here is "parity unpinned".
 """
 
-from . import e4m3, paged, attention  # noqa: F401
+from . import e4m3, paged, attention, acceptance  # noqa: F401

@@ -17,21 +17,38 @@ orders:
   4c..4c+3 hold slots 2c, 2c+1, 2c+8, 2c+9.
 * ``"dim"`` (head-dim-major): ``uint8[P, Hkv, D, ps]``; the same as
   ``"grp16"`` when ps = 16.
+* ``"ksw"`` (token-major, chunk-permuted): ``uint8[P, Hkv, ps, 128]`` -- the
+  token-major order with each token row cut into eight 16-byte chunks, and
+  chunk j of slot s stored at chunk position ``j XOR (s % 8)``.  The K pages
+  use it when D = 128 (the permutation is the 128-byte swizzle of the
+  tensor-core operand layout, so a page copied verbatim is ready to use);
+  with D = 64 K pages are plain ``"tok"``.
 
 The block table is the fixed-size-block pool of the Atlas deep-dive
 (ainews.cool, "Memory architecture" paragraph: KV blocks preallocated in
 fixed sizes); the FP8 codes are those of the GB10 page's "paged FP8 KV cache"
-(ainews.surl.tw).  The two layouts are spelled out only in :func:`slot_of`,
-:func:`_store` and :func:`gather_codes`.
+(ainews.surl.tw).  The layouts are spelled out only in :func:`slot_of`,
+:func:`ksw_chunk`, :func:`_store` and :func:`gather_codes`.
 """
 
 import numpy as np
 
 from . import e4m3
 
-LAYOUTS = ("tok", "grp16", "dim")
+LAYOUTS = ("tok", "grp16", "dim", "ksw")
 GROUP = 16
 GROUP_POS = np.array([4 * ((t % 8) // 2) + 2 * (t // 8) + t % 2 for t in range(GROUP)])
+
+
+def ksw_chunk(slot: int, j: int) -> int:
+    """Chunk position of logical 16-byte chunk ``j`` of slot ``slot`` in the
+    ``"ksw"`` order."""
+    return j ^ (slot % 8)
+
+
+def k_layout(head_dim: int) -> str:
+    """In-page order of the K pages for a head dimension."""
+    return "ksw" if head_dim == 128 else "tok"
 
 
 def slot_of(block_table, b: int, pos: int, page_size: int):
@@ -47,6 +64,10 @@ def _store(out, page, slot, codes, layout):
         out[page, :, slot // GROUP, :, GROUP_POS[slot % GROUP]] = codes
     elif layout == "dim":
         out[page, :, :, slot] = codes
+    elif layout == "ksw":
+        for j in range(8):
+            c = ksw_chunk(slot, j)
+            out[page, :, slot, 16 * c:16 * c + 16] = codes[:, 16 * j:16 * j + 16]
     else:
         raise ValueError(layout)
 
@@ -86,6 +107,13 @@ def gather_codes(pages, block_table, b: int, length: int, page_size: int, layout
         seq = seq.reshape(seq.shape[0], seq.shape[1] * GROUP, seq.shape[3], seq.shape[4])
     elif layout == "dim":                     # [n_pages, Hkv, D, ps]
         seq = blocks.transpose(0, 3, 1, 2)
+    elif layout == "ksw":                     # [n_pages, Hkv, ps, 128], chunks permuted
+        un = np.empty_like(blocks)
+        for slot in range(blocks.shape[2]):
+            for j in range(8):
+                c = ksw_chunk(slot, j)
+                un[:, :, slot, 16 * j:16 * j + 16] = blocks[:, :, slot, 16 * c:16 * c + 16]
+        seq = un.transpose(0, 2, 1, 3)
     else:
         raise ValueError(layout)
     hkv = seq.shape[2]

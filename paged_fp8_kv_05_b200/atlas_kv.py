@@ -34,6 +34,8 @@ OPT_PARTITION = 4
 OPT_ROWS_PER_CTA = 5
 OPT_WAIT_LIMIT_US = 6
 OPT_TEST_SKIP_UNIT = 7
+OPT_KERNEL = 8
+KERNEL_AUTO, KERNEL_WARP_MMA, KERNEL_TC = 0, 1, 2
 PLAN_FIELDS = ("split_tokens", "num_splits", "kernel", "rows_per_cta", "row_blocks",
                "launches", "grid_ctas")
 
@@ -70,6 +72,8 @@ _SIGNATURES = [
       _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_plan", ctypes.c_int,
      [_c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.POINTER(_c_i32), _c_i32]),
+    ("atlas_mtp_greedy_accept", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr]),
     ("atlas_get_device_error", ctypes.c_int, [_c_ptr, _c_ptr, ctypes.POINTER(_c_i32)]),
 ]
 for _name, _res, _args in _SIGNATURES:
@@ -120,7 +124,8 @@ class KVPool:
 
     ``atlas_kv_pool_create`` on caller-owned torch buffers; the buffers live
     as long as this object.  ``k_pages`` is uint8
-    ``[num_pages, num_kv_heads, page_size, head_dim]`` (token-major) and
+    ``[num_pages, num_kv_heads, page_size, head_dim]`` (token-major; with
+    head_dim 128 the 16-byte chunk j of slot s sits at chunk j ^ (s % 8)) and
     ``v_pages`` uint8 ``[num_pages, num_kv_heads, page_size // 16, head_dim, 16]``
     (16-slot groups, head-dim-major inside a group).
     """
@@ -254,6 +259,29 @@ def atlas_paged_gqa_decode_noalloc(q, k_pages, v_pages, k_scale, v_scale, block_
                                                float(sm_scale), _ptr(out), _stream(stream)),
            "atlas_paged_gqa_decode_noalloc")
     return out
+
+
+def atlas_mtp_greedy_accept(pool: KVPool, logits, drafts, targets=None, n_accepted=None,
+                            next_token=None, stream=None):
+    """Greedy MTP acceptance.  ``logits``: ``[B, K + 1, V]`` float32 or bf16;
+    ``drafts``: int32 ``[B, K]``.  Returns ``(n_accepted [B], next_token [B],
+    targets [B, K + 1])`` (int32 device tensors)."""
+    assert logits.dim() == 3 and logits.is_contiguous() and drafts.is_contiguous()
+    B, K1, V = (int(x) for x in logits.shape)
+    assert tuple(drafts.shape) == (B, K1 - 1) and drafts.dtype == torch.int32
+    dtype = {torch.float32: ATLAS_DTYPE_F32, torch.bfloat16: ATLAS_DTYPE_BF16}[logits.dtype]
+    dev = logits.device
+    if targets is None:
+        targets = torch.empty(B, K1, dtype=torch.int32, device=dev)
+    if n_accepted is None:
+        n_accepted = torch.empty(B, dtype=torch.int32, device=dev)
+    if next_token is None:
+        next_token = torch.empty(B, dtype=torch.int32, device=dev)
+    _check(_lib.atlas_mtp_greedy_accept(pool.handle, _ptr(logits), dtype, B, K1 - 1, V,
+                                        _ptr(drafts), _ptr(targets), _ptr(n_accepted),
+                                        _ptr(next_token), _stream(stream)),
+           "atlas_mtp_greedy_accept")
+    return n_accepted, next_token, targets
 
 
 def atlas_paged_gqa_decode_plan(pool: KVPool, batch, num_q_heads, q_len, max_seq_len) -> dict:

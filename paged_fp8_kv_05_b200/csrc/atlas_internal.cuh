@@ -67,6 +67,12 @@ constexpr unsigned long long kDefaultWaitLimitNs = 200ull * 1000 * 1000;
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
 
+// Greedy MTP acceptance: one CTA per logits row; counters: int32 [batch],
+// zero before the launch and left zero.
+cudaError_t launch_mtp_accept(const void* logits, int dtype, int batch, int num_drafts, int vocab,
+                              const int32_t* drafts, int32_t* targets, int32_t* n_accepted,
+                              int32_t* next_token, int32_t* counters, cudaStream_t stream);
+
 // Launch shape of the decode kernel for one call (A1).  A segment is
 // (sequence, KV head, row group of rows_per_cta query rows); a unit is 32 KV
 // tokens of a segment.
@@ -95,6 +101,73 @@ struct DecodeLaunch {
 };
 
 constexpr int kMaxUnitsPerCta = 1024;  // bounds the per-CTA unit table in shared memory
+
+// Which decode kernel serves a call: the FP8 warp-MMA kernel (mma.sync, any
+// row count, head_dim 64 or 128) or the 5th-generation tensor-core kernel
+// (tcgen05.mma with accumulators in tensor memory, head_dim 128, blocks of 64
+// query rows).  Automatic: tcgen05 when head_dim is 128 and a KV head has at
+// least kTcMinRows query rows (q_len * G), where QK^T and PV are real
+// contractions; the warp-MMA kernel otherwise.
+enum { kKernelAuto = 0, kKernelWarpMma = 1, kKernelTc = 2 };
+constexpr int kTcMinRows = 16;
+
+inline bool use_tc_kernel(int kernel, int head_dim, int q_len, int G) {
+  if (kernel == kKernelWarpMma) return false;
+  if (kernel == kKernelTc) return true;
+  return head_dim == 128 && q_len * G >= kTcMinRows;
+}
+
+// Launch plan of the tensor-core kernel: grid partition (CTA = one split of a
+// (sequence, KV head, 64-row block) segment, splits of a multiple of 128
+// tokens), two resident CTAs per SM.  split_tokens > 0 overrides the split
+// length (rounded up to a multiple of 128).
+inline DecodeLaunch plan_decode_tc(int B, int Hq, int Hkv, int q_len, int max_seq_len, int sms,
+                                   int split_tokens, int stages_override, int waves = 1) {
+  DecodeLaunch L;
+  L.waves = waves < 1 ? 1 : waves;
+  const int R = q_len * (Hq / Hkv);
+  L.rows_per_warp = 16;
+  L.rbg = 4;
+  L.rows_per_cta = 64;
+  L.row_blocks = (R + 63) / 64;
+  L.stages = stages_override > 0 ? stages_override : 2;
+  L.segs = (long long)B * Hkv * L.row_blocks;
+  L.units_max = L.segs * (((long long)max_seq_len + 31) / 32);
+  L.grid_mode = 1;
+  const long long resident = (long long)sms * 2;
+  long long T;
+  if (split_tokens > 0) {
+    T = (split_tokens + 127) / 128 * 128;
+  } else {
+    // as the warp-MMA grid partition: splits for two to four waves of
+    // resident CTAs if every sequence were max_seq_len long, but not under
+    // 2048 tokens unless one wave needs shorter ones; multiple of 128 in
+    // [256, 8192]
+    const long long segs = L.segs > 0 ? L.segs : 1;
+    auto split_for = [&](long long ctas) {
+      long long want = (ctas + segs - 1) / segs;
+      if (want < 1) want = 1;
+      const long long t = ((long long)max_seq_len + want - 1) / want;
+      return (t + 127) / 128 * 128;
+    };
+    const long long one_wave = split_for(resident * L.waves);
+    const long long two_waves = split_for(2 * resident * L.waves);
+    T = 128;
+    while (2 * T <= two_waves) T *= 2;
+    const long long lo = one_wave < 2048 ? one_wave : 2048;
+    if (T < lo) T = lo;
+    if (T < 256) T = 256;
+    if (T > 8192) T = 8192;
+  }
+  L.split_tokens = (int)T;
+  L.num_splits = (int)(((long long)max_seq_len + T - 1) / T);
+  if (L.num_splits < 1) L.num_splits = 1;
+  L.grid = L.segs * L.num_splits;
+  L.max_units = (int)((T + 31) / 32);
+  L.max_portions = 1;
+  L.slots = L.num_splits > 1 ? L.segs * L.num_splits : 0;
+  return L;
+}
 
 // Resident CTAs per SM the kernel is built for (its __launch_bounds__).
 inline int decode_target_occupancy(int rows_per_warp, int rbg) {
@@ -192,6 +265,12 @@ inline DecodeLaunch plan_decode(int B, int Hq, int Hkv, int q_len, int max_seq_l
 cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg, int stages,
                               long long grid, cudaStream_t stream);
 
+// Tensor-core decode kernel (head_dim 128): 1-D grid of `grid` CTAs, one per
+// (segment, split); stages 2 or 3.
+cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
+                             cudaStream_t stream);
+size_t decode_tc_smem_bytes(int stages, int split_tokens);
+
 // Dynamic shared memory of one decode CTA (rows = min(rows_per_cta, q_len * G)).
 size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units,
                              int max_portions);
@@ -270,13 +349,23 @@ __device__ __forceinline__ uint4 quantize16_e4m3(const float (&x)[16], float sca
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 16-byte chunk position of head dims [16j, 16j + 16) of K slot `slot`: with
+// D = 128 each 128-byte token row is stored with its eight chunks permuted,
+// chunk j at j XOR (slot % 8) -- the 128-byte swizzle of the tensor-core
+// operand layout, so a 16-token piece copied verbatim into 1024-byte-aligned
+// shared memory is a ready K-major operand; with D = 64 rows are plain.
+__device__ __forceinline__ int k_chunk_pos(int D, int slot, int j) {
+  return D == 128 ? (j ^ (slot & 7)) : j;
+}
+
 // Store 16 codes of head dims [16j, 16j + 16) of token slot `slot` of a head's
-// page.  K pages are token-major [P][Hkv][ps][D]; V pages are 16-slot groups,
-// head-dim-major inside a group, [P][Hkv][ps/16][D][16], with slot t of a group
-// at byte 4*((t%8)/2) + 2*(t/8) + t%2.
+// page.  K pages are token-major [P][Hkv][ps][D] (chunks placed by
+// k_chunk_pos); V pages are 16-slot groups, head-dim-major inside a group,
+// [P][Hkv][ps/16][D][16], with slot t of a group at byte
+// 4*((t%8)/2) + 2*(t/8) + t%2.
 __device__ __forceinline__ void store16_k(uint8_t* k_pages, size_t head_page, int D, int ps,
                                           int slot, int j, uint4 codes) {
-  uint8_t* dst = k_pages + (head_page * ps + slot) * D + 16 * j;
+  uint8_t* dst = k_pages + (head_page * ps + slot) * D + 16 * k_chunk_pos(D, slot, j);
   *reinterpret_cast<uint4*>(dst) = codes;
 }
 __device__ __forceinline__ void store16_v(uint8_t* v_pages, size_t head_page, int D, int ps,

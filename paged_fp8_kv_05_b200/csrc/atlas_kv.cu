@@ -22,6 +22,7 @@ struct atlas_kv_pool {
   int32_t waves_override;
   int32_t partition_override;
   int32_t rows_override;
+  int32_t kernel_override; // atlas::kKernel*
   int32_t wait_limit_us;   // 0: the default limit of every bounded wait
   int32_t test_skip_unit;  // -1: normal; >= 0: lost-copy injection (tests only)
   size_t counters_bytes;  // largest counter block any accepted call uses
@@ -76,7 +77,13 @@ WsLayout ws_layout(const atlas::DecodeLaunch& L, int head_dim) {
 // "block size adapted to sequence length and architecture" of the Atlas
 // deep-dive's attention paragraph.
 atlas::DecodeLaunch make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
-                              int max_seq_len, int sms, bool fit) {
+                              int max_seq_len, int sms, bool fit, bool* tc) {
+  *tc = atlas::use_tc_kernel(pool->kernel_override, pool->head_dim, q_len,
+                             num_q_heads / pool->num_kv_heads);
+  if (*tc)
+    return atlas::plan_decode_tc(batch, num_q_heads, pool->num_kv_heads, q_len, max_seq_len, sms,
+                                 pool->split_override, pool->stages_override,
+                                 pool->waves_override > 0 ? pool->waves_override : 1);
   atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, pool->num_kv_heads, q_len,
                                              max_seq_len, sms, pool->split_override,
                                              pool->stages_override, pool->partition_override,
@@ -137,6 +144,14 @@ size_t atlas_kv_workspace_bytes(int32_t max_batch, int32_t max_q_len, int32_t nu
         const size_t t = ws_layout(L, head_dim).total;
         if (t > need) need = t;
       }
+    // the tensor-core kernel's plans (head_dim 128)
+    if (head_dim == 128)
+      for (int split : {0, min_split_tokens}) {
+        const atlas::DecodeLaunch L =
+            atlas::plan_decode_tc(max_batch, num_q_heads, num_kv_heads, ql, msl, sms, split, 0);
+        const size_t t = ws_layout(L, head_dim).total;
+        if (t > need) need = t;
+      }
     // the counter block of the finest row grouping (4 rows per block)
     const atlas::DecodeLaunch L4 = atlas::plan_decode(max_batch, num_q_heads, num_kv_heads, ql,
                                                       msl, sms, 0, 0, atlas::kPartitionGrid, 1, 4);
@@ -191,6 +206,7 @@ atlas_status_t atlas_kv_pool_create(atlas_kv_pool_t** out, int32_t num_pages, in
   p->waves_override = 0;
   p->partition_override = 0;
   p->rows_override = 0;
+  p->kernel_override = 0;
   p->wait_limit_us = 0;
   p->test_skip_unit = -1;
   p->counters_bytes = counters_bytes;
@@ -233,6 +249,11 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
       if (value != 0 && value != 4 && value != 8 && value != 16 && value != 32 && value != 64)
         return ATLAS_ERR_INVALID_ARG;
       pool->rows_override = value;
+      return ATLAS_OK;
+    case ATLAS_OPT_KERNEL:
+      if (value < 0 || value > 2) return ATLAS_ERR_INVALID_ARG;
+      if (value == atlas::kKernelTc && pool->head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
+      pool->kernel_override = value;
       return ATLAS_OK;
     case ATLAS_OPT_WAIT_LIMIT_US:
       if (value < 0 || value > 10 * 1000 * 1000) return ATLAS_ERR_INVALID_ARG;
@@ -297,15 +318,17 @@ atlas_status_t atlas_paged_gqa_decode_plan(const atlas_kv_pool_t* pool, int32_t 
   if (!plan || n < 0) return ATLAS_ERR_INVALID_ARG;
   const bool dev = device_present();
   const int sms = dev ? device_sm_count() : kDefaultSms;
-  const atlas::DecodeLaunch L = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, dev);
+  bool tc = false;
+  const atlas::DecodeLaunch L =
+      make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, dev, &tc);
   long long spread = L.num_splits;  // grid partition: splits per segment
   if (!L.grid_mode) {  // balanced: most ranges a max-length segment can meet
     const long long seg_units = ((long long)max_seq_len + 31) / 32;
     spread = 1 + (seg_units - 1 + L.max_units - 1) / L.max_units;
     if (spread > L.grid) spread = L.grid;
   }
-  const int32_t split = pool->split_override > 0 ? pool->split_override : L.split_tokens;
-  const int32_t f[ATLAS_PLAN_FIELDS] = {split, (int32_t)spread, L.grid_mode ? 1 : 2,
+  const int32_t split = (!tc && pool->split_override > 0) ? pool->split_override : L.split_tokens;
+  const int32_t f[ATLAS_PLAN_FIELDS] = {split, (int32_t)spread, tc ? 3 : L.grid_mode ? 1 : 2,
                                         L.rows_per_cta, L.row_blocks, 1,
                                         (int32_t)(L.grid > 0x7FFFFFFF ? 0x7FFFFFFF : L.grid)};
   for (int i = 0; i < n && i < ATLAS_PLAN_FIELDS; ++i) plan[i] = f[i];
@@ -335,7 +358,9 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
     return ATLAS_ERR_INVALID_ARG;
 
   const int sms = device_sm_count();
-  const atlas::DecodeLaunch L = make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true);
+  bool tc = false;
+  const atlas::DecodeLaunch L =
+      make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true, &tc);
   const WsLayout ws = ws_layout(L, pool->head_dim);
   if (ws.total > pool->workspace_bytes) return ATLAS_ERR_WORKSPACE;
   if (L.grid > 0x7FFFFFFFLL) return ATLAS_ERR_UNSUPPORTED;
@@ -378,8 +403,10 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.wait_limit_ns = pool->wait_limit_us > 0 ? 1000ull * pool->wait_limit_us
                                             : atlas::kDefaultWaitLimitNs;
   p.test_skip_unit = pool->test_skip_unit;
-  cudaError_t e = atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid,
-                                           static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      tc ? atlas::launch_decode_tc(p, L.stages, L.grid, static_cast<cudaStream_t>(stream))
+         : atlas::launch_decode_fp8(p, L.rows_per_warp, L.rbg, L.stages, L.grid,
+                                    static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
 
@@ -412,6 +439,25 @@ atlas_status_t atlas_paged_gqa_append_decode(const atlas_kv_pool_t* pool, const 
   return decode_impl(pool, q, pool->k_pages, pool->v_pages, pool->k_scale, pool->v_scale,
                      block_table, max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len,
                      max_seq_len, sm_scale, out, k_new, v_new, dtype, stream);
+}
+
+atlas_status_t atlas_mtp_greedy_accept(const atlas_kv_pool_t* pool, const void* logits,
+                                       int32_t dtype, int32_t batch, int32_t num_drafts,
+                                       int32_t vocab, const int32_t* drafts, int32_t* targets,
+                                       int32_t* n_accepted, int32_t* next_token, void* stream) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (batch < 0 || batch > pool->max_batch || num_drafts < 0 || vocab < 1)
+    return ATLAS_ERR_INVALID_ARG;
+  if (dtype != ATLAS_DTYPE_F32 && dtype != ATLAS_DTYPE_BF16) return ATLAS_ERR_INVALID_ARG;
+  if (batch == 0) return ATLAS_OK;
+  if (!logits || !targets || !n_accepted || !next_token || (num_drafts > 0 && !drafts))
+    return ATLAS_ERR_INVALID_ARG;
+  if ((size_t)batch * sizeof(int32_t) > pool->counters_bytes) return ATLAS_ERR_WORKSPACE;
+  int32_t* counters = reinterpret_cast<int32_t*>(pool->workspace + kAlign);
+  cudaError_t e = atlas::launch_mtp_accept(logits, dtype, batch, num_drafts, vocab, drafts,
+                                           targets, n_accepted, next_token, counters,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
 
 atlas_status_t atlas_get_device_error(const atlas_kv_pool_t* pool, void* stream, int32_t* code) {

@@ -529,19 +529,18 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   float acc[MT][NT][4];
 
   // this lane's K operand words of one 16-token K tile: rows g8 and g8 + 8,
-  // 16-byte chunks 4j + c (D = 128: odd rows fetch their chunks in the other
-  // order, which keeps the 8 lanes of each shared-memory phase on distinct banks)
+  // 16-byte chunks 4j + c.  D = 128: the pages store chunk j of slot s at
+  // j XOR (s % 8), and a 16-token piece starts at a multiple of 16 slots, so
+  // row g8 (+ 8) finds logical chunk 4j + c at (4j + c) ^ g8 -- which also
+  // puts the 8 lanes of each shared-memory phase on distinct banks
   auto load_k = [&](const uint8_t* kt, uint4 (&kr)[2][NCH]) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int row = g8 + 8 * t;
       if constexpr (D == 128) {
-        const int ja = g8 & 1;
         const uint8_t* rb = kt + row * 128;
-        const uint4 x0 = *reinterpret_cast<const uint4*>(rb + ((4 * ja + c) << 4));
-        const uint4 x1 = *reinterpret_cast<const uint4*>(rb + ((4 * (1 - ja) + c) << 4));
-        kr[t][0] = ja ? x1 : x0;
-        kr[t][1] = ja ? x0 : x1;
+        kr[t][0] = *reinterpret_cast<const uint4*>(rb + (((0 + c) ^ g8) << 4));
+        kr[t][1] = *reinterpret_cast<const uint4*>(rb + (((4 + c) ^ g8) << 4));
       } else {
         kr[t][0] = *reinterpret_cast<const uint4*>(kt + row * 64 + (c << 4));
       }

@@ -280,3 +280,35 @@ def workload_tag(index: int) -> str:
     c = CONFIGS[index]
     return (f"{c['name']}: B={c['batch']} Hq={c['num_q_heads']} Hkv={c['num_kv_heads']} "
             f"D={c['head_dim']} ps={c['page_size']} q_len={c['q_len']} lengths={c['lengths']}")
+
+
+def make_verify_logits(*, batch, num_drafts, vocab, seed=0, dtype=torch.bfloat16, ties=False):
+    """Synthetic verify-step logits and MTP drafts for greedy acceptance.
+
+    ``logits`` ``[B, K + 1, V]``: N(0, 1) draws (rounded to ``dtype``) with one
+    planted token per row whose logit is 8.0 (far above the draws); with
+    ``ties`` a second token of every row gets the same 8.0.  ``drafts``
+    int32 ``[B, K]``: each sequence draws an agreement length a in 0..K; draft
+    i is the row's planted token for i < a, and a different token at i = a
+    (the tokens after it are random).  Pure input construction: the planted
+    tokens are chosen, never computed from the logits."""
+    s_log, s_tok, s_len, s_rest = np.random.SeedSequence(seed).spawn(4)
+    K1 = num_drafts + 1
+    x = np.random.default_rng(s_log).standard_normal((batch, K1, vocab), dtype=np.float32)
+    rt = np.random.default_rng(s_tok)
+    planted = rt.integers(0, vocab, size=(batch, K1))
+    rows = np.arange(batch)[:, None], np.arange(K1)[None, :]
+    x[rows[0], rows[1], planted] = 8.0
+    second = None
+    if ties:
+        second = rt.integers(0, vocab, size=(batch, K1))
+        x[rows[0], rows[1], second] = 8.0
+    a = np.random.default_rng(s_len).integers(0, num_drafts + 1, size=batch)
+    rr = np.random.default_rng(s_rest)
+    drafts = rr.integers(0, vocab, size=(batch, max(num_drafts, 0))).astype(np.int32)
+    for b in range(batch):
+        drafts[b, :a[b]] = planted[b, :a[b]]
+        if a[b] < num_drafts and vocab > 1:
+            drafts[b, a[b]] = (planted[b, a[b]] + 1 + rr.integers(0, vocab - 1)) % vocab
+    logits = torch.from_numpy(x).to(dtype)
+    return logits, drafts, dict(planted=planted, agree=a, second=second)

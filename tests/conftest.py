@@ -37,6 +37,7 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     if not PARITY_LOG:
         return
     tr = terminalreporter
-    tr.write_sep("-", "parity against the float64 oracle (bound: max-abs 1e-2, rel-L2 5e-3)")
+    tr.write_sep("-", "parity against the float64 oracle (bound: |d| <= max(1e-2, 2^-8 |ref|) "
+                      "per element, rel-L2 5e-3)")
     for case, max_abs, rel in PARITY_LOG:
         tr.write_line(f"{case:<72s} max-abs {max_abs:.3e}  rel-L2 {rel:.3e}")

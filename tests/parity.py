@@ -6,10 +6,17 @@ import numpy as np
 
 from oracle import attention, e4m3, paged
 
-# Tolerance of the decode / verify output against the float64 oracle:
-# max-abs <= 1e-2 and relative L2 <= 5e-3 over the compared rows.  The bf16
-# store alone contributes up to 2^-9 relative per element.
+# Tolerance of the decode / verify output against the float64 oracle (bf16
+# out, f32 softmax): relative L2 <= 5e-3 over the compared rows, and per
+# element |got - ref| <= max(1e-2, 2^-8 |ref|).  The 1e-2 absolute bound is
+# the stated one for unit-scale outputs; bf16 keeps 8 significant bits, so
+# the correctly rounded output of a value of magnitude >= 4 (half an ulp is
+# then 2^-6 or more) can already be more than 1e-2 away.  2^-8 |ref| bounds
+# that rounding (at most 2^-9 |ref|) with room for the f32 arithmetic; it
+# only exceeds 1e-2 where |ref| > 2.56, so unit-scale outputs keep the plain
+# 1e-2 bound.
 MAX_ABS = 1e-2
+REL_ELEM = 2.0 ** -8
 REL_L2 = 5e-3
 
 
@@ -17,7 +24,8 @@ def oracle_pages(w, which):
     """Token-major uint8 pages ``[P, Hkv, ps, D]`` the oracle expects after
     every token of every sequence of workload ``w`` is appended, and the mask
     of written (page, head, slot) triples.  (The GPU keeps V in 16-slot
-    groups; tests bring it to token-major with :func:`v_token_major`.)"""
+    groups and, with D = 128, K rows chunk-permuted; tests bring them to
+    token-major with :func:`v_token_major` and :func:`k_token_major`.)"""
     P, Hkv, ps, D = w.num_pages, w.num_kv_heads, w.page_size, w.head_dim
     pages = np.zeros((P, Hkv, ps, D), np.uint8)
     written = np.zeros((P, Hkv, ps), bool)
@@ -31,6 +39,21 @@ def oracle_pages(w, which):
         pages[pg, :, t % ps, :] = codes
         written[pg, :, t % ps] = True
     return pages, written
+
+
+def k_token_major(k):
+    """GPU K pages ``[P, Hkv, ps, D]`` (chunk-permuted rows when D = 128) ->
+    plain token-major ``[P, Hkv, ps, D]``."""
+    k = np.asarray(k)
+    P, H, ps, D = k.shape
+    if paged.k_layout(D) == "tok":
+        return k
+    out = np.empty_like(k)
+    for s in range(ps):
+        for j in range(D // 16):
+            c = paged.ksw_chunk(s, j)
+            out[:, :, s, 16 * j:16 * j + 16] = k[:, :, s, 16 * c:16 * c + 16]
+    return out
 
 
 def v_token_major(v):
@@ -85,12 +108,28 @@ def record_parity(case, max_abs, rel):
     PARITY_LOG.append((case, float(max_abs), float(rel)))
 
 
+def elementwise_excess(got, ref):
+    """Largest ratio |got - ref| / max(MAX_ABS, REL_ELEM |ref|) over the finite
+    rows of ref (<= 1 passes)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    sel = np.isfinite(ref)
+    if not sel.any():
+        return 0.0
+    d = np.abs(got[sel] - ref[sel])
+    allowed = np.maximum(MAX_ABS, REL_ELEM * np.abs(ref[sel]))
+    return float(np.max(d / allowed))
+
+
 def assert_close(got, ref, what=""):
     max_abs, rel = errors(got, ref)
     assert np.all(np.isfinite(np.asarray(got, np.float64)[np.isfinite(ref)])), f"{what}: non-finite output"
-    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {max_abs:.3g}, rel-L2 {rel:.3g}"
+    excess = elementwise_excess(got, ref)
+    assert excess <= 1.0 and rel <= REL_L2, (
+        f"{what}: max-abs {max_abs:.3g} ({excess:.3g} of the per-element bound), rel-L2 {rel:.3g}")
     return max_abs, rel
 
 
-__all__ = ["oracle_pages", "oracle_decode", "errors", "assert_close", "record_parity",
-           "PARITY_LOG", "MAX_ABS", "REL_L2", "paged"]
+__all__ = ["oracle_pages", "oracle_decode", "k_token_major", "v_token_major", "errors",
+           "assert_close", "elementwise_excess", "record_parity", "PARITY_LOG", "MAX_ABS",
+           "REL_ELEM", "REL_L2", "paged"]

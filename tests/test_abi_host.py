@@ -239,10 +239,13 @@ def _plan_on_148_sms(B, Hq, Hkv, D, ps, q_len, max_seq_len, P=1024):
     ((32, 32, 8, 128, 16, 1, 4096), dict(kernel=1, split_tokens=2048, grid_ctas=512, rows_per_cta=4)),
     # long context: 32 segments; two waves -> 4736 tokens, rounded down to 4096
     ((4, 32, 8, 128, 16, 1, 131072), dict(kernel=1, split_tokens=4096, num_splits=32, grid_ctas=1024)),
-    # MTP verify: 1024 segments already fill the GPU; one split of the whole length
-    ((128, 40, 8, 128, 16, 5, 1152), dict(kernel=1, split_tokens=1152, grid_ctas=1024, rows_per_cta=32)),
-    # MQA with 64 rows: one K/V stream per CTA -> balanced ranges, 2 per SM
-    ((256, 64, 1, 128, 64, 1, 8192), dict(kernel=2, grid_ctas=296, rows_per_cta=64)),
+    # MTP verify, 25 rows per KV head: the tensor-core kernel; 1024 segments of
+    # one 64-row block already fill the GPU -> one split of the whole length
+    ((128, 40, 8, 128, 16, 5, 1152), dict(kernel=3, split_tokens=1152, grid_ctas=1024, rows_per_cta=64)),
+    # MQA with 64 rows: the tensor-core kernel; two waves of 296 CTA slots over
+    # 256 segments -> 2816 tokens, rounded down to 2048: 4 splits
+    ((256, 64, 1, 128, 64, 1, 8192), dict(kernel=3, split_tokens=2048, num_splits=4, grid_ctas=1024,
+                                          rows_per_cta=64)),
 ])
 def test_automatic_plan_of_the_named_shapes(shape, want):
     plan = _plan_on_148_sms(*shape)

@@ -8,7 +8,7 @@ import torch
 from oracle import e4m3, paged
 from paged_fp8_kv_05_b200 import build, workloads
 
-from parity import oracle_pages, v_token_major
+from parity import k_token_major, oracle_pages, v_token_major
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +36,8 @@ def test_cache_fill_bit_exact(ak, cfg):
         got = dev.cpu().numpy()
         if which == "v":                                 # V pages: 16-slot groups
             got = v_token_major(got)
+        else:                                            # K rows: chunk-permuted at D = 128
+            got = k_token_major(got)
         assert np.array_equal(got[written], want[written]), f"{which}: codes differ"
         assert np.all(got[~written] == 0x7F), f"{which}: stray writes"
 
@@ -110,7 +112,7 @@ def test_bf16_input_and_ragged_positions(ak):
     assert pool.device_error() == 0
     init_k = np.full((P, Hkv, ps, D), 0x7F, np.uint8)
     init_v = np.full((P, Hkv, ps // 16, D, 16), 0x7F, np.uint8)
-    want_k = paged.append(init_k, x_exact, ks, table, start, ps, layout="tok")
+    want_k = paged.append(init_k, x_exact, ks, table, start, ps, layout=paged.k_layout(D))
     want_v = paged.append(init_v, (vt.float().cpu().numpy()), vs, table, start, ps, layout="grp16")
     assert np.array_equal(pool.k_pages.cpu().numpy(), want_k)
     assert np.array_equal(pool.v_pages.cpu().numpy(), want_v)

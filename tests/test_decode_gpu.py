@@ -36,18 +36,25 @@ def _oracle_named(cfg, w):
     return _ORACLE[cfg]
 
 
-# partition 0 = automatic (grid for 0-2, balanced for the MQA case 4); the
-# other partition of configs 1 and 4 is checked too
-@pytest.mark.parametrize("cfg,partition", [(0, 0), (1, 0), (2, 0), (4, 0), (1, 2), (4, 1)])
-def test_named_workload_full_output(ak, cfg, partition):
+# kernel 0 = automatic (the tensor-core kernel for the verify and MQA
+# workloads 2 and 4, the warp-MMA kernel for 0 and 1); the warp-MMA kernel is
+# also checked on 2 and 4, in both of its partitions where they differ
+# (partition 0 = automatic: grid, or balanced when one K/V stream serves a CTA)
+@pytest.mark.parametrize("cfg,kernel,partition", [
+    (0, 0, 0), (1, 0, 0), (2, 0, 0), (4, 0, 0),
+    (1, 1, 2), (2, 1, 0), (4, 1, 0), (4, 1, 1)])
+def test_named_workload_full_output(ak, cfg, kernel, partition):
     w = workloads.config_workload(cfg)
     dw = _dw(w)
+    dw.pool.set_option(ak.OPT_KERNEL, kernel)
     dw.pool.set_option(ak.OPT_PARTITION, partition)
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
     ref = _oracle_named(cfg, w)
-    max_abs, rel = assert_close(got, ref, f"config {cfg}, partition {partition}")
-    record_parity(f"config {cfg}, partition {partition}", max_abs, rel)
+    plan = dw.plan()
+    what = f"config {cfg}, kernel {plan['kernel']} (option {kernel}), partition {partition}"
+    max_abs, rel = assert_close(got, ref, what)
+    record_parity(what, max_abs, rel)
     print(f"config {cfg}: max-abs {max_abs:.3e} rel-L2 {rel:.3e} plan {dw.plan()}")
 
 
@@ -95,10 +102,12 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("kernel", [0, 1])
 @pytest.mark.parametrize("case", EDGE)
-def test_edge_cases(ak, case):
+def test_edge_cases(ak, case, kernel):
     w = _case(*case)
     dw = _dw(w)
+    dw.pool.set_option(ak.OPT_KERNEL, kernel)
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
     assert_close(got, oracle_decode(w), f"edge {case}")
@@ -117,6 +126,7 @@ def test_both_partitions(ak, case, split, partition):
     segment cut into many parts, merged by the CTA that finishes it last)."""
     w = _case(*case, seed=11)
     dw = _dw(w, min_split_tokens=64)
+    dw.pool.set_option(ak.OPT_KERNEL, ak.KERNEL_WARP_MMA)
     dw.pool.set_option(ak.OPT_PARTITION, partition)
     dw.pool.set_split_tokens(split)
     plan = dw.plan()
@@ -180,6 +190,7 @@ def test_mtp_rows_ignore_later_drafts(ak):
     q_len = 5
     w = _case(2, 40, 8, 128, 16, [130, 77], q_len, seed=8)
     dw = _dw(w)
+    dw.pool.set_option(ak.OPT_KERNEL, ak.KERNEL_WARP_MMA)
     base = dw.decode(out=torch.empty_like(dw.q)).clone()
     for i in range(q_len - 1):
         kp = dw.pool.k_pages.clone()
@@ -256,6 +267,7 @@ def test_lost_copy_times_out_and_the_library_stays_usable(ak):
     same pool must be clean and match everywhere."""
     w = _case(4, 32, 8, 128, 16, [700, 1500, 64, 300], 1, seed=12)
     dw = _dw(w)
+    dw.pool.set_option(ak.OPT_KERNEL, ak.KERNEL_WARP_MMA)
     dw.pool.set_option(ak.OPT_PARTITION, 1)
     dw.pool.set_option(ak.OPT_WAIT_LIMIT_US, 1000)
     dw.pool.set_option(ak.OPT_TEST_SKIP_UNIT, 1)

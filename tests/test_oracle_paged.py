@@ -134,3 +134,31 @@ def test_grp16_layout_groups_sixteen_slots_head_dim_major():
     t = paged.append(tok, new, sc, table, np.array([40]), ps, layout="tok")
     for s in range(ps):
         assert np.array_equal(a[:, :, s // 16, :, where[s % 16]], t[:, :, s, :])
+
+
+def test_ksw_layout_permutes_sixteen_byte_chunks_by_slot():
+    """Explicit construction: byte 16 * (j ^ (s % 8)) + k of slot s holds
+    logical byte 16 * j + k (the 128-byte swizzle of a 128-byte row)."""
+    rng = np.random.default_rng(29)
+    P, Hkv, ps, D = 4, 2, 32, 128
+    tok = rng.integers(0, 256, (P, Hkv, ps, D), dtype=np.uint8)
+    sw = np.empty_like(tok)
+    for s_ in range(ps):
+        for j in range(8):
+            dst = (j ^ (s_ % 8)) * 16
+            sw[:, :, s_, dst:dst + 16] = tok[:, :, s_, 16 * j:16 * j + 16]
+    # slot 0 is unpermuted; slot 3 moves chunk 0 to position 3 and chunk 3 to 0
+    assert np.array_equal(sw[:, :, 0], tok[:, :, 0])
+    assert np.array_equal(sw[:, :, 3, 48:64], tok[:, :, 3, 0:16])
+    assert np.array_equal(sw[:, :, 3, 0:16], tok[:, :, 3, 48:64])
+    table = np.array([[2, 0, 3], [1, -1, -1]], dtype=np.int32)
+    for b, L in [(0, 70), (1, 32), (0, 1), (1, 17)]:
+        assert np.array_equal(paged.gather_codes(tok, table, b, L, ps, "tok"),
+                              paged.gather_codes(sw, table, b, L, ps, "ksw"))
+    new = rng.standard_normal((1, 9, Hkv, D)).astype(np.float32)
+    sc = np.array([0.02, 0.05], np.float32)
+    a = paged.append(sw, new, sc, table, np.array([28]), ps, layout="ksw")
+    t = paged.append(tok, new, sc, table, np.array([28]), ps, layout="tok")
+    assert np.array_equal(paged.gather_codes(a, table, 0, 37, ps, "ksw"),
+                          paged.gather_codes(t, table, 0, 37, ps, "tok"))
+    assert paged.k_layout(128) == "ksw" and paged.k_layout(64) == "tok"

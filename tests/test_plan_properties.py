@@ -43,13 +43,14 @@ shapes = st.tuples(
     st.sampled_from([64, 128]),               # head_dim
     st.sampled_from([0, 1, 2]),               # partition option
     st.sampled_from([0, 64, 128, 448, 2048, 8192]),  # split override
+    st.sampled_from([0, 1, 2]),               # kernel option (auto, warp-MMA, tcgen05)
 )
 
 
 @settings(max_examples=300, deadline=None)
 @given(shapes)
 def test_plan_covers_every_token_and_fits_its_workspace(shape):
-    B, Hkv, G, q_len, msl, D, part, split = shape
+    B, Hkv, G, q_len, msl, D, part, split, kern = shape
     Hq = Hkv * G
     msl = max(msl, q_len)
     h = ctypes.c_void_p()
@@ -59,12 +60,34 @@ def test_plan_covers_every_token_and_fits_its_workspace(shape):
     try:
         assert ak._lib.atlas_kv_pool_set_option(h, ak.OPT_PARTITION, part) == ak.ATLAS_OK
         assert ak._lib.atlas_kv_pool_set_split_tokens(h, split) == ak.ATLAS_OK
+        st_k = ak._lib.atlas_kv_pool_set_option(h, ak.OPT_KERNEL, kern)
+        if kern == 2 and D != 128:
+            assert st_k == ak.ATLAS_ERR_UNSUPPORTED
+            return
+        assert st_k == ak.ATLAS_OK
         p = _plan(h, B, Hq, q_len, msl)
     finally:
         ak._lib.atlas_kv_pool_destroy(h)
 
     R = q_len * G
     rc, rb = p["rows_per_cta"], p["row_blocks"]
+    tc = kern == 2 or (kern == 0 and D == 128 and R >= 16)
+    assert (p["kernel"] == 3) == tc
+    if tc:                                     # tensor-core kernel: 64-row blocks, grid
+        T = p["split_tokens"]
+        segs = B * Hkv * math.ceil(R / 64)
+        assert rc == 64 and rb == math.ceil(R / 64)
+        assert T % 128 == 0 and p["num_splits"] * T >= msl and (p["num_splits"] - 1) * T < msl
+        if split:
+            assert T == (split + 127) // 128 * 128
+        else:
+            assert 256 <= T <= 8192
+        assert p["grid_ctas"] == segs * p["num_splits"]
+        slots = segs * p["num_splits"] if p["num_splits"] > 1 else 0
+        need = ALIGN + _align(segs * 4) + _align(slots * rc * 4) + _align(slots * rc * D * 4)
+        have = ak.atlas_kv_workspace_bytes(B, q_len, Hq, Hkv, D, msl, 64)
+        assert have >= need, (p, have, need)
+        return
     # the row block is the smallest of 4, 8, 16, 32, 64 holding R rows (or 64)
     assert rc in (4, 8, 16, 32, 64) and rb == math.ceil(R / rc)
     assert rc == 64 or rc >= R

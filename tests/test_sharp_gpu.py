@@ -17,9 +17,10 @@ oracle finishes in seconds):
   along the context, so that row's scores grow by ~1.4 (base 2) per 32-token
   unit and its softmax reference has to move on nearly every unit.
 
-Each case runs in both partitions, with the automatic split length and with
-64-token splits (segments cut into many parts, merged by log-sum-exp), and
-is compared element by element with the oracle at max-abs 1e-2, rel-L2 5e-3.
+Each case runs on the warp-MMA kernel in both partitions and on the
+tensor-core kernel, with the automatic split length and with 128-token
+splits (segments cut into many parts, merged by log-sum-exp), and is
+compared element by element with the oracle at max-abs 1e-2, rel-L2 5e-3.
 """
 
 import functools
@@ -70,18 +71,25 @@ def ak():
     return atlas_kv
 
 
-@pytest.mark.parametrize("split", [0, 64])
-@pytest.mark.parametrize("partition", [1, 2])
+# (ATLAS_OPT_KERNEL, ATLAS_OPT_PARTITION): warp-MMA kernel in its grid and
+# balanced partitions, and the tensor-core kernel
+KERNELS = {"warp-grid": (1, 1), "warp-balanced": (1, 2), "tcgen05": (2, 0)}
+
+
+@pytest.mark.parametrize("split", [0, 128])
+@pytest.mark.parametrize("kernel", list(KERNELS))
 @pytest.mark.parametrize("variant", list(VARIANTS))
 @pytest.mark.parametrize("shape", list(SHAPES))
-def test_sharp_attention(ak, shape, variant, partition, split):
+def test_sharp_attention(ak, shape, variant, kernel, split):
     from paged_fp8_kv_05_b200.device_cache import DeviceWorkload
     w = _workload(shape, variant)
     dw = DeviceWorkload(w, min_split_tokens=64)
+    kern, partition = KERNELS[kernel]
+    dw.pool.set_option(ak.OPT_KERNEL, kern)
     dw.pool.set_option(ak.OPT_PARTITION, partition)
     dw.pool.set_split_tokens(split)
     got = dw.decode().float().cpu().numpy()
     assert dw.pool.device_error() == 0
-    case = f"sharp {shape} {variant} partition {partition} split {split or 'auto'}"
+    case = f"sharp {shape} {variant} {kernel} split {split or 'auto'}"
     max_abs, rel = assert_close(got, _oracle(shape, variant), case)
     record_parity(case, max_abs, rel)
