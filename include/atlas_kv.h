@@ -222,6 +222,34 @@ ATLAS_API atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const 
                                    void* stream);
 
 /*
+ * Fused rotary embedding + FP8 quantise + paged append from the QKV
+ * projection output of the new tokens (Atlas deep-dive, ainews.cool, "Kernel
+ * fusion" paragraph: per-block steps fused into one kernel).  qkv: device
+ * bf16 [batch][n_new][num_q_heads + 2 * num_kv_heads][head_dim] (per token:
+ * the query heads, then the key heads, then the value heads), 16-byte
+ * aligned.  cos_sin: device float32 [max_pos][head_dim], cos of the rotation
+ * angles in columns 0 .. head_dim/2 - 1 and sin in the rest.  Token t of
+ * sequence b has position start_pos[b] + t (device int32 [batch]).  Query and
+ * key heads are rotated "rotate half" style (element i < head_dim/2 with
+ * i + head_dim/2: out[i] = x[i] c - x[i+D/2] s, out[i+D/2] = x[i+D/2] c +
+ * x[i] s) in float32 with every product and sum rounded separately; the
+ * rotated queries are written to q_out (device bf16
+ * [batch][n_new][num_q_heads][head_dim], round to nearest even), the rotated
+ * keys and the values are quantised and written into the pool's pages exactly
+ * as atlas_fp8_kv_append does.  Bit-exact with that definition.  A token whose
+ * position is outside [0, max_pos) is skipped entirely (its q_out rows are
+ * left unwritten); a position past the block table or a bad page id skips
+ * that token's K and V rows; both flag ATLAS_DEVERR_APPEND.  batch == 0 or
+ * n_new == 0 is a no-op.
+ */
+ATLAS_API atlas_status_t atlas_rope_fp8_kv_append(const atlas_kv_pool_t* pool, const void* qkv,
+                                                  int32_t num_q_heads, const float* cos_sin,
+                                                  int32_t max_pos, const int32_t* block_table,
+                                                  int32_t max_blocks_per_seq,
+                                                  const int32_t* start_pos, int32_t batch,
+                                                  int32_t n_new, void* q_out, void* stream);
+
+/*
  * Paged decode (q_len == 1) / MTP-verify (q_len > 1) grouped-query attention.
  * q: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
  * k_pages / v_pages: the pool's page arrays (or arrays of identical shape).
@@ -249,6 +277,26 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, con
                                       int32_t batch, int32_t num_q_heads, int32_t q_len,
                                       int32_t max_seq_len, float sm_scale, void* out,
                                       void* stream);
+
+/*
+ * Ragged verify and chunked prefill over the paged cache: the same attention
+ * as atlas_paged_gqa_decode, with a number of new rows per sequence (GB10
+ * page: MTP verification at concurrency 1-128, where sequences verify
+ * different numbers of drafts; a prefill chunk is the same with many rows).
+ * cu_q_lens: device int32 [batch + 1], packed row offsets (cu_q_lens[0] = 0,
+ * non-decreasing); sequence b owns rows cu_q_lens[b] .. cu_q_lens[b+1] - 1 of
+ * q and out (device bf16 [cu_q_lens[batch]][num_q_heads][head_dim]), its
+ * q_len_b = cu_q_lens[b+1] - cu_q_lens[b] may be 0 (nothing written).  New row
+ * i of sequence b sees key positions t <= seq_lens[b] - q_len_b + i.
+ * max_q_len: host upper bound of every q_len_b (<= the pool's max_q_len; it
+ * sizes the row blocks).  The warp-MMA kernel runs the grid partition here.
+ * Other arguments and errors as atlas_paged_gqa_decode.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_decode_varlen(
+    const atlas_kv_pool_t* pool, const void* q, const int32_t* cu_q_lens, const void* k_pages,
+    const void* v_pages, const float* k_scale, const float* v_scale, const int32_t* block_table,
+    int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+    int32_t max_q_len, int32_t max_seq_len, float sm_scale, void* out, void* stream);
 
 /*
  * One decode / verify step in one kernel: the FP8 append of the q_len new

@@ -79,3 +79,43 @@ def paged_gqa_decode(q, k_pages, v_pages, k_scale, v_scale, block_table,
                 out[b, :, hq, :] = attend(q[b, :, hq, :], K[:, h, :], V[:, h, :],
                                           limits, sm_scale)
     return out
+
+
+def paged_gqa_decode_varlen(q, cu_q_lens, k_pages, v_pages, k_scale, v_scale, block_table,
+                            seq_lens, page_size, sm_scale=None, sequences=None,
+                            k_layout="tok", v_layout="tok"):
+    """Ragged verify / chunked prefill: sequence b has its own number of new
+    rows ``q_len_b = cu_q_lens[b + 1] - cu_q_lens[b]`` (packed: rows
+    ``cu_q_lens[b] .. cu_q_lens[b + 1] - 1`` of ``q``), and new row i of it
+    sees key positions ``t <= L_b - q_len_b + i`` (the GB10 page's MTP under
+    concurrency: sequences verify different numbers of drafts; a prefill
+    chunk is the same with many rows).  ``q`` float64 ``[total, Hq, D]``;
+    returns float64 ``[total, Hq, D]`` (rows of skipped sequences NaN)."""
+    q = np.asarray(q, dtype=np.float64)
+    cu = np.asarray(cu_q_lens, dtype=np.int64)
+    total, Hq, D = q.shape
+    assert cu[0] == 0 and cu[-1] == total and np.all(np.diff(cu) >= 0)
+    Hkv = np.asarray(k_pages).shape[1]
+    assert Hq % Hkv == 0, "Hq must be a multiple of Hkv"
+    G = Hq // Hkv
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / math.sqrt(D)
+    out = np.full((total, Hq, D), np.nan)
+    B = len(cu) - 1
+    for b in (range(B) if sequences is None else sequences):
+        L = int(seq_lens[b])
+        ql = int(cu[b + 1] - cu[b])
+        if ql == 0:
+            continue
+        if L < ql:
+            raise ValueError(f"sequence {b}: seq_len {L} < q_len {ql}")
+        K = paged.gather_dequant(k_pages, k_scale, block_table, b, L, page_size, k_layout)
+        V = paged.gather_dequant(v_pages, v_scale, block_table, b, L, page_size, v_layout)
+        limits = [L - ql + i for i in range(ql)]
+        rows = slice(cu[b], cu[b + 1])
+        for h in range(Hkv):
+            for g in range(G):
+                hq = h * G + g
+                out[rows, hq, :] = attend(q[rows, hq, :], K[:, h, :], V[:, h, :], limits,
+                                          sm_scale)
+    return out

@@ -72,6 +72,12 @@ _SIGNATURES = [
       _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_plan", ctypes.c_int,
      [_c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.POINTER(_c_i32), _c_i32]),
+    ("atlas_paged_gqa_decode_varlen", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32,
+      _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
+    ("atlas_rope_fp8_kv_append", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_ptr,
+      _c_ptr]),
     ("atlas_mtp_greedy_accept", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr]),
     ("atlas_get_device_error", ctypes.c_int, [_c_ptr, _c_ptr, ctypes.POINTER(_c_i32)]),
@@ -259,6 +265,49 @@ def atlas_paged_gqa_decode_noalloc(q, k_pages, v_pages, k_scale, v_scale, block_
                                                float(sm_scale), _ptr(out), _stream(stream)),
            "atlas_paged_gqa_decode_noalloc")
     return out
+
+
+def atlas_paged_gqa_decode_varlen(pool: KVPool, q, cu_q_lens, block_table, seq_lens,
+                                  max_q_len, max_seq_len, out=None, sm_scale=0.0, k_pages=None,
+                                  v_pages=None, k_scale=None, v_scale=None, stream=None):
+    """Ragged verify / chunked prefill.  ``q``: bf16 ``[total_rows, Hq, D]``
+    packed by ``cu_q_lens`` (int32 ``[B + 1]``); returns ``out`` (same shape)."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.dim() == 3
+    assert cu_q_lens.dtype == torch.int32 and block_table.is_contiguous()
+    B = int(cu_q_lens.shape[0]) - 1
+    Hq = int(q.shape[1])
+    if out is None:
+        out = torch.empty_like(q)
+    kp = pool.k_pages if k_pages is None else k_pages
+    vp = pool.v_pages if v_pages is None else v_pages
+    ks = pool.k_scale if k_scale is None else k_scale
+    vs = pool.v_scale if v_scale is None else v_scale
+    _check(_lib.atlas_paged_gqa_decode_varlen(pool.handle, _ptr(q), _ptr(cu_q_lens), _ptr(kp),
+                                              _ptr(vp), _ptr(ks), _ptr(vs), _ptr(block_table),
+                                              int(block_table.shape[1]), _ptr(seq_lens), B, Hq,
+                                              int(max_q_len), int(max_seq_len), float(sm_scale),
+                                              _ptr(out), _stream(stream)),
+           "atlas_paged_gqa_decode_varlen")
+    return out
+
+
+def atlas_rope_fp8_kv_append(pool: KVPool, qkv, num_q_heads, cos_sin, block_table, start_pos,
+                             q_out=None, stream=None):
+    """Rotate Q and K of the new tokens, quantise and append K and V.
+    ``qkv``: bf16 ``[B, n_new, Hq + 2 Hkv, D]``; ``cos_sin``: float32
+    ``[max_pos, D]``.  Returns the rotated queries ``q_out`` (bf16
+    ``[B, n_new, Hq, D]``)."""
+    assert qkv.dtype == torch.bfloat16 and qkv.is_contiguous() and cos_sin.is_contiguous()
+    assert cos_sin.dtype == torch.float32 and block_table.is_contiguous()
+    B, n_new, heads, D = (int(x) for x in qkv.shape)
+    if q_out is None:
+        q_out = torch.empty(B, n_new, num_q_heads, D, dtype=torch.bfloat16, device=qkv.device)
+    _check(_lib.atlas_rope_fp8_kv_append(pool.handle, _ptr(qkv), num_q_heads, _ptr(cos_sin),
+                                         int(cos_sin.shape[0]), _ptr(block_table),
+                                         int(block_table.shape[1]), _ptr(start_pos), B, n_new,
+                                         _ptr(q_out), _stream(stream)),
+           "atlas_rope_fp8_kv_append")
+    return q_out
 
 
 def atlas_mtp_greedy_accept(pool: KVPool, logits, drafts, targets=None, n_accepted=None,

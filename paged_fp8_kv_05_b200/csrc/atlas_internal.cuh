@@ -38,6 +38,8 @@ struct DecodeParams {
   const float* v_scale;
   const int32_t* block_table; // [B][max_blocks]
   const int32_t* seq_lens;    // [B]
+  const int32_t* cu_q;        // nullptr: q_len rows per sequence; else [B + 1] packed row
+                              // offsets (q, out are [cu_q[B]][Hq][D], q_len = the largest)
   __nv_bfloat16* out;         // [B][q_len][Hq][D]
   float* part_o;              // [slots][rows_per_cta][D]  (partials of cut segments)
   float* part_lse;            // [slots][rows_per_cta]     (log2-domain LSE)
@@ -66,6 +68,23 @@ struct DecodeParams {
 constexpr unsigned long long kDefaultWaitLimitNs = 200ull * 1000 * 1000;
 
 cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t stream);
+
+struct RopeAppendParams {
+  const __nv_bfloat16* qkv;   // [B][n_new][Hq + 2 Hkv][D]: query, key, value heads
+  const float* cos_sin;       // [max_pos][D]: cos in columns 0..D/2-1, sin in D/2..D-1
+  int max_pos;
+  __nv_bfloat16* q_out;       // [B][n_new][Hq][D]: rotated queries
+  uint8_t* k_pages;
+  uint8_t* v_pages;
+  const float* k_scale;       // [Hkv]
+  const float* v_scale;
+  const int32_t* block_table; // [B][max_blocks]
+  const int32_t* start_pos;   // [B]
+  int32_t* err;
+  int batch, n_new, Hq, Hkv, D, ps, num_pages, max_blocks;
+};
+
+cudaError_t launch_rope_append(const RopeAppendParams& p, cudaStream_t stream);
 
 // Greedy MTP acceptance: one CTA per logits row; counters: int32 [batch],
 // zero before the launch and left zero.

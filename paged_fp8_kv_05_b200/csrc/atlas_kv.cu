@@ -77,16 +77,20 @@ WsLayout ws_layout(const atlas::DecodeLaunch& L, int head_dim) {
 // "block size adapted to sequence length and architecture" of the Atlas
 // deep-dive's attention paragraph.
 atlas::DecodeLaunch make_plan(const atlas_kv_pool* pool, int batch, int num_q_heads, int q_len,
-                              int max_seq_len, int sms, bool fit, bool* tc) {
+                              int max_seq_len, int sms, bool fit, bool* tc, bool varlen = false) {
   *tc = atlas::use_tc_kernel(pool->kernel_override, pool->head_dim, q_len,
                              num_q_heads / pool->num_kv_heads);
   if (*tc)
     return atlas::plan_decode_tc(batch, num_q_heads, pool->num_kv_heads, q_len, max_seq_len, sms,
                                  pool->split_override, pool->stages_override,
                                  pool->waves_override > 0 ? pool->waves_override : 1);
+  // ragged q_len: the grid partition (a CTA serves one segment, so row blocks
+  // past a sequence's rows cost nothing)
   atlas::DecodeLaunch L = atlas::plan_decode(batch, num_q_heads, pool->num_kv_heads, q_len,
                                              max_seq_len, sms, pool->split_override,
-                                             pool->stages_override, pool->partition_override,
+                                             pool->stages_override,
+                                             varlen ? atlas::kPartitionGrid
+                                                    : pool->partition_override,
                                              pool->waves_override > 0 ? pool->waves_override : 1,
                                              pool->rows_override);
   if (fit && pool->split_override == 0 && !L.grid_mode) {
@@ -299,6 +303,44 @@ atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_ne
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
 
+atlas_status_t atlas_rope_fp8_kv_append(const atlas_kv_pool_t* pool, const void* qkv,
+                                        int32_t num_q_heads, const float* cos_sin,
+                                        int32_t max_pos, const int32_t* block_table,
+                                        int32_t max_blocks_per_seq, const int32_t* start_pos,
+                                        int32_t batch, int32_t n_new, void* q_out,
+                                        void* stream) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (batch < 0 || n_new < 0 || max_blocks_per_seq < 1 || num_q_heads < 1 || max_pos < 1)
+    return ATLAS_ERR_INVALID_ARG;
+  if (num_q_heads % pool->num_kv_heads != 0) return ATLAS_ERR_INVALID_ARG;
+  if (batch == 0 || n_new == 0) return ATLAS_OK;
+  if (!qkv || !cos_sin || !block_table || !start_pos || !q_out) return ATLAS_ERR_INVALID_ARG;
+  if (!aligned(qkv, 16) || !aligned(cos_sin, 16) || !aligned(q_out, 16))
+    return ATLAS_ERR_INVALID_ARG;
+  atlas::RopeAppendParams p{};
+  p.qkv = static_cast<const __nv_bfloat16*>(qkv);
+  p.cos_sin = cos_sin;
+  p.max_pos = max_pos;
+  p.q_out = static_cast<__nv_bfloat16*>(q_out);
+  p.k_pages = pool->k_pages;
+  p.v_pages = pool->v_pages;
+  p.k_scale = pool->k_scale;
+  p.v_scale = pool->v_scale;
+  p.block_table = block_table;
+  p.start_pos = start_pos;
+  p.err = reinterpret_cast<int32_t*>(pool->workspace);
+  p.batch = batch;
+  p.n_new = n_new;
+  p.Hq = num_q_heads;
+  p.Hkv = pool->num_kv_heads;
+  p.D = pool->head_dim;
+  p.ps = pool->page_size;
+  p.num_pages = pool->num_pages;
+  p.max_blocks = max_blocks_per_seq;
+  cudaError_t e = atlas::launch_rope_append(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
 static atlas_status_t check_decode_shape(const atlas_kv_pool_t* pool, int32_t batch,
                                          int32_t num_q_heads, int32_t q_len,
                                          int32_t max_seq_len) {
@@ -344,7 +386,7 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
                                   const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
                                   int32_t q_len, int32_t max_seq_len, float sm_scale, void* out,
                                   const void* k_new, const void* v_new, int32_t new_dtype,
-                                  void* stream) {
+                                  void* stream, const int32_t* cu_q = nullptr) {
   atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
   if (st != ATLAS_OK) return st;
   if (max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
@@ -360,7 +402,7 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   const int sms = device_sm_count();
   bool tc = false;
   const atlas::DecodeLaunch L =
-      make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true, &tc);
+      make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true, &tc, cu_q != nullptr);
   const WsLayout ws = ws_layout(L, pool->head_dim);
   if (ws.total > pool->workspace_bytes) return ATLAS_ERR_WORKSPACE;
   if (L.grid > 0x7FFFFFFFLL) return ATLAS_ERR_UNSUPPORTED;
@@ -373,6 +415,7 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.v_scale = v_scale;
   p.block_table = block_table;
   p.seq_lens = seq_lens;
+  p.cu_q = cu_q;
   p.out = static_cast<__nv_bfloat16*>(out);
   uint8_t* wsp = pool->workspace;
   p.err = reinterpret_cast<int32_t*>(wsp);
@@ -423,6 +466,20 @@ atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q
   return decode_impl(pool, q, k_pages, v_pages, k_scale, v_scale, block_table,
                      max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len, max_seq_len,
                      sm_scale, out, nullptr, nullptr, ATLAS_DTYPE_F32, stream);
+}
+
+atlas_status_t atlas_paged_gqa_decode_varlen(const atlas_kv_pool_t* pool, const void* q,
+                                             const int32_t* cu_q_lens, const void* k_pages,
+                                             const void* v_pages, const float* k_scale,
+                                             const float* v_scale, const int32_t* block_table,
+                                             int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                             int32_t batch, int32_t num_q_heads,
+                                             int32_t max_q_len, int32_t max_seq_len,
+                                             float sm_scale, void* out, void* stream) {
+  if (batch > 0 && !cu_q_lens) return ATLAS_ERR_INVALID_ARG;
+  return decode_impl(pool, q, k_pages, v_pages, k_scale, v_scale, block_table,
+                     max_blocks_per_seq, seq_lens, batch, num_q_heads, max_q_len, max_seq_len,
+                     sm_scale, out, nullptr, nullptr, ATLAS_DTYPE_F32, stream, cu_q_lens);
 }
 
 atlas_status_t atlas_paged_gqa_append_decode(const atlas_kv_pool_t* pool, const void* k_new,

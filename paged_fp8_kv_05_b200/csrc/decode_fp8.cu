@@ -169,6 +169,7 @@ struct Portion {
   int k0;               // first unit of the portion inside the CTA's range
   int slot0;            // first partial slot of the segment
   int my, n_parts;      // this portion's part index and the segment's part count
+  int ql, qb;           // the sequence's new rows and its first packed q / out row
   float k_scale, v_scale;  // the KV head's dequantisation scales
 };
 
@@ -241,8 +242,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   constexpr int TILE = 16 * D;           // one 16-token K piece or V^T piece
   constexpr int STAGE = 4 * TILE;        // K_A, K_B, V_A, V_B
 
-  const int Rtot = p.q_len * p.G;
-  const int rows_max = min(RC, Rtot);    // rows of the fullest row group
+  const int Rmax = p.q_len * p.G;        // p.q_len: the largest q_len of any sequence
+  const int rows_max = min(RC, Rmax);    // rows of the fullest row group
   extern __shared__ __align__(16) uint8_t smem[];
   const SmemPlan sp = smem_plan(D, S, NSTREAM, rows_max, p.max_units, p.max_portions);
   uint8_t* ring = smem;
@@ -266,8 +267,16 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   const int cid = blockIdx.x, G = gridDim.x;
   const int RB = p.row_blocks;          // row groups per (b, h)
   const int Hs = p.Hkv * RB;            // segments per sequence
-  auto valid_len = [&](int L) {
-    return L >= p.q_len && L <= p.max_blocks * p.ps && L <= p.max_seq_len;
+  // new rows of sequence b and its first row in q / out: uniform q_len, or
+  // per sequence from the packed offsets cu_q (ragged verify, prefill chunks)
+  auto qlen_of = [&](int b) {
+    return p.cu_q ? __ldg(p.cu_q + b + 1) - __ldg(p.cu_q + b) : p.q_len;
+  };
+  auto qbase_of = [&](int b) { return p.cu_q ? __ldg(p.cu_q + b) : b * p.q_len; };
+  // a sequence with rows is served when q_len <= L <= the table row and the
+  // host's max_seq_len; one with no rows (ragged only) is skipped silently
+  auto valid_len = [&](int L, int ql) {
+    return ql >= 1 && L >= ql && L <= p.max_blocks * p.ps && L <= p.max_seq_len;
   };
   auto units_of = [&](int L) { return (L + kUnit - 1) / kUnit; };
 
@@ -275,10 +284,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   // or the host's max_seq_len): zero all their rows and flag them; one CTA per b
   for (int bb = cid; bb < p.B; bb += G) {
     const int L = __ldg(p.seq_lens + bb);
-    if (valid_len(L)) continue;
+    const int ql = qlen_of(bb);
+    if (ql == 0 || valid_len(L, ql)) continue;
     if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
-    const size_t n = (size_t)p.q_len * p.Hq * D;
-    __nv_bfloat16* o = p.out + (size_t)bb * n;
+    const size_t n = (size_t)max(ql, 0) * p.Hq * D;
+    __nv_bfloat16* o = p.out + (size_t)qbase_of(bb) * p.Hq * D;
     for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
   }
 
@@ -293,12 +303,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const int split = cid % p.num_splits, sg = cid / p.num_splits;
     const int b = sg / Hs, seg = sg % Hs;
     const int L = __ldg(p.seq_lens + b);
-    if (!valid_len(L)) return;  // CTA-uniform; its rows were zeroed above
+    const int ql = qlen_of(b);
+    if (!valid_len(L, ql)) return;  // CTA-uniform; its rows were zeroed above
+    if ((seg % RB) * RC >= ql * p.G) return;  // a row block past this sequence's rows
     const int t_begin = split * p.split_tokens;
     if (t_begin >= L) return;
     if (tid == 0) {
       Portion P;
       P.b = b; P.seg = seg; P.L = L; P.ua = t_begin / kUnit; P.k0 = 0;
+      P.ql = ql; P.qb = qbase_of(b);
       P.slot0 = sg * p.num_splits;
       P.my = split;
       P.n_parts = (L + p.split_tokens - 1) / p.split_tokens;
@@ -316,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     unsigned long long mine = 0;
     for (int bb = bb0; bb < bb1; ++bb) {
       const int L = __ldg(p.seq_lens + bb);
-      if (valid_len(L)) mine += (unsigned long long)Hs * units_of(L);
+      if (valid_len(L, qlen_of(bb))) mine += (unsigned long long)Hs * units_of(L);
     }
     unsigned long long total = 0;
     const unsigned long long first = block_exclusive_scan(mine, s_scan, total);
@@ -339,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       long long P = (long long)first;
       for (int bb = bb0; bb < bb1 && P < u1; ++bb) {
         const int L = __ldg(p.seq_lens + bb);
-        if (!valid_len(L)) continue;
+        if (!valid_len(L, qlen_of(bb))) continue;
         const int n = units_of(L);
         const long long size = (long long)Hs * n;
         if (P + size > u0) {
@@ -357,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       long long P = (long long)first;
       for (int bb = bb0; bb < bb1 && P < u1; ++bb) {
         const int L = __ldg(p.seq_lens + bb);
-        if (!valid_len(L)) continue;
+        if (!valid_len(L, qlen_of(bb))) continue;
         const int n = units_of(L);
         const long long size = (long long)Hs * n;
         if (P + size > u0) {
@@ -368,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
             const long long a = max(s0, u0);
             Portion Q;
             Q.b = bb; Q.seg = seg; Q.L = L;
+            Q.ql = qlen_of(bb); Q.qb = qbase_of(bb);
             Q.ua = (int)(a - s0);
             Q.k0 = (int)(a - u0);
             const int c_first = owner_cta(s0, U, Ge);
@@ -393,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
   auto prefetch_q = [&](int pi) {
     const Portion P = s_port[pi];
     const int h = P.seg / RB, r0 = (P.seg % RB) * RC;
-    const int rows = min(RC, Rtot - r0);
+    const int rows = max(0, min(RC, P.ql * p.G - r0));
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     __nv_bfloat16* dst = s_q + (size_t)(pi % kQBuf) * rows_max * D;
     for (int idx = tid; idx < rows * CPR; idx += kThreads) {
@@ -401,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       const int r = r0 + lr;
       const int i = r / p.G, hq = h * p.G + r % p.G;
       cp_async16(dst + lr * D + ch * 8,
-                 p.q + (((size_t)P.b * p.q_len + i) * p.Hq + hq) * D + ch * 8);
+                 p.q + (((size_t)P.qb + i) * p.Hq + hq) * D + ch * 8);
     }
     cp_async_commit();
   };
@@ -446,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       const Portion P = s_port[pi];
       const int L = P.L;
       const int h = P.seg / RB;
-      const int first_new_pos = L - p.q_len;
+      const int first_new_pos = L - P.ql;
       const int a0 = max(kUnit * P.ua, first_new_pos);
       const int a1 = min(kUnit * (P.ua + port_end(pi) - P.k0), L);
       const int n_tok = a1 - a0;
@@ -464,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         }
         float x[16];
         load16_as_f32(which ? p.v_new : p.k_new,
-                      (((size_t)P.b * p.q_len + (pos - first_new_pos)) * p.Hkv + h) * D + 16 * j,
+                      (((size_t)P.qb + (pos - first_new_pos)) * p.Hkv + h) * D + 16 * j,
                       p.new_dtype, x);
         const uint4 codes = quantize16_e4m3(x, which ? P.v_scale : P.k_scale);
         const size_t head_page = (size_t)page * p.Hkv + h;
@@ -721,8 +735,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const Portion P = s_port[pi];
     const int b = P.b, seg = P.seg, L = P.L;
     const int h = seg / RB, rg = seg % RB;
+    const int Rtot = P.ql * p.G;           // this sequence's query rows per KV head
     const int cta_row0 = rg * RC;
-    const int rows_cta = min(RC, Rtot - cta_row0);
+    const int rows_cta = max(0, min(RC, Rtot - cta_row0));
     const int row0 = cta_row0 + rbw * RW;  // this warp's first row
     const int kb = P.k0, ke = port_end(pi);
     const bool whole = (P.n_parts == 1);
@@ -808,11 +823,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         // the row of accumulator column 2c + e (PK: columns c and c ^ 2 are one row)
         const int rl = PK ? 2 * (c & 1) + e : 8 * nt + 2 * c + e;
         const int r = row0 + rl;
-        lim[nt][e] = (r < Rtot) ? (L - p.q_len + r / p.G) : (L - 1);
+        lim[nt][e] = (r < Rtot) ? (L - P.ql + r / p.G) : (L - 1);
         const float a = __shfl_sync(kFull, alpha_row[nt], 4 * (rl - 8 * nt));
         scale2[nt][e] = kscale / a;
       }
-    min_lim = L - p.q_len + row0 / p.G;
+    min_lim = L - P.ql + row0 / p.G;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       m_run[nt][0] = m_run[nt][1] = -INFINITY;
@@ -897,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
             const float den = l_full[nt][e];
             const float inv = den > 0.f ? 1.f / den : 0.f;
             if (whole) {
-              __nv_bfloat16* orow = p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * D;
+              __nv_bfloat16* orow = p.out + (((size_t)P.qb + i) * p.Hq + hq) * D;
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
                 orow[16 * mt + g8] = __float2bfloat16_rn(acc[mt][nt][e] * inv * vs);
@@ -956,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
         const int r = cta_row0 + lr;
         const int i = r / p.G, hq = h * p.G + r % p.G;
         if (whole) {
-          p.out[(((size_t)b * p.q_len + i) * p.Hq + hq) * D + d] =
+          p.out[(((size_t)P.qb + i) * p.Hq + hq) * D + d] =
               __float2bfloat16_rn(den > 0.f ? num / den * vs : 0.f);
         } else {
           p.part_o[(slot * RC + lr) * D + d] = (den > 0.f) ? num / den : 0.f;
@@ -990,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
     const Portion P = s_port[q == 0 ? cut0 : cut1];
     const int seg_idx = P.b * Hs + P.seg;
     const int h = P.seg / RB, cta_row0 = (P.seg % RB) * RC;
-    const int rows_cta = min(RC, Rtot - cta_row0);
+    const int rows_cta = max(0, min(RC, P.ql * p.G - cta_row0));
     int32_t* counter = p.counters + seg_idx;
     __syncthreads();  // every thread's partial stores are fenced; s_is_last is free
     if (tid == 0) s_is_last = (atomicAdd(counter, 1) == P.n_parts - 1);
@@ -1034,7 +1049,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
       const float inv = den > 0.f ? vs / den : 0.f;
       const int r = cta_row0 + lr;
       const int i = r / p.G, hq = h * p.G + r % p.G;
-      __nv_bfloat16* dst = p.out + (((size_t)P.b * p.q_len + i) * p.Hq + hq) * D + d0;
+      __nv_bfloat16* dst = p.out + (((size_t)P.qb + i) * p.Hq + hq) * D + d0;
       const __nv_bfloat162 lo = __floats2bfloat162_rn(o4.x * inv, o4.y * inv);
       const __nv_bfloat162 hi = __floats2bfloat162_rn(o4.z * inv, o4.w * inv);
       uint2 pk;

@@ -268,18 +268,24 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cid = blockIdx.x, G = gridDim.x;
   const int RB = p.row_blocks, Hs = p.Hkv * RB;
-  const int Rtot = p.q_len * p.G;
-  auto valid_len = [&](int L) {
-    return L >= p.q_len && L <= p.max_blocks * p.ps && L <= p.max_seq_len;
+  // new rows of sequence b and its first row in q / out: uniform q_len, or
+  // per sequence from the packed offsets cu_q (ragged verify, prefill chunks)
+  auto qlen_of = [&](int bb) {
+    return p.cu_q ? __ldg(p.cu_q + bb + 1) - __ldg(p.cu_q + bb) : p.q_len;
+  };
+  auto qbase_of = [&](int bb) { return p.cu_q ? __ldg(p.cu_q + bb) : bb * p.q_len; };
+  auto valid_len = [&](int L, int ql) {
+    return ql >= 1 && L >= ql && L <= p.max_blocks * p.ps && L <= p.max_seq_len;
   };
 
   // ---- invalid sequences: zero all their rows and flag them; one CTA per b
   for (int bb = cid; bb < p.B; bb += G) {
     const int L = __ldg(p.seq_lens + bb);
-    if (valid_len(L)) continue;
+    const int ql = qlen_of(bb);
+    if (ql == 0 || valid_len(L, ql)) continue;
     if (tid == 0) atomicOr(p.err, ATLAS_DEVERR_SEQ_LEN);
-    const size_t n = (size_t)p.q_len * p.Hq * kD;
-    __nv_bfloat16* o = p.out + (size_t)bb * n;
+    const size_t n = (size_t)max(ql, 0) * p.Hq * kD;
+    __nv_bfloat16* o = p.out + (size_t)qbase_of(bb) * p.Hq * kD;
     for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
   }
 
@@ -287,7 +293,10 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   const int split = cid % p.num_splits, sg = cid / p.num_splits;
   const int b = sg / Hs, seg = sg % Hs, h = seg / RB, rb = seg % RB;
   const int L = __ldg(p.seq_lens + b);
-  if (!valid_len(L)) return;               // CTA-uniform; rows zeroed above
+  const int q_len = qlen_of(b), q_base = qbase_of(b);
+  if (!valid_len(L, q_len)) return;        // CTA-uniform; rows zeroed above
+  const int Rtot = q_len * p.G;            // this sequence's query rows per KV head
+  if (rb * kRows >= Rtot) return;          // a row block past this sequence's rows
   const int T = p.split_tokens;
   const int t_begin = split * T;
   if (t_begin >= L) return;
@@ -303,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   // ---- A0, fused append: the step's new tokens that fall in this split are
   // quantised and stored before any bulk copy reads the pages
   if (p.k_new != nullptr) {
-    const int first_new = L - p.q_len;
+    const int first_new = L - q_len;
     const int a0 = max(t_begin, first_new);
     const int n_new = t_end - a0;
     if (n_new > 0) {
@@ -319,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         }
         float x[16];
         load16_as_f32(which ? p.v_new : p.k_new,
-                      (((size_t)b * p.q_len + (pos - first_new)) * p.Hkv + h) * kD + 16 * j,
+                      (((size_t)q_base + (pos - first_new)) * p.Hkv + h) * kD + 16 * j,
                       p.new_dtype, x);
         const uint4 codes = quantize16_e4m3(x, which ? v_scale : k_scale);
         const size_t head_page = (size_t)page * p.Hkv + h;
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     if (r < rows) {
       const int i = rr / p.G, hq = h * p.G + rr % p.G;
       const uint4* src = reinterpret_cast<const uint4*>(
-          p.q + (((size_t)b * p.q_len + i) * p.Hq + hq) * kD + 64 * my_half);
+          p.q + (((size_t)q_base + i) * p.Hq + hq) * kD + 64 * my_half);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 w = __ldg(src + c);
@@ -371,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           x[8 * c + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
         }
       }
-      row_lim = L - p.q_len + i;
+      row_lim = L - q_len + i;
     } else {
 #pragma unroll
       for (int k = 0; k < 64; ++k) x[k] = 0.f;
@@ -705,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         if (whole) {
           const float inv = den > 0.f ? v_scale / den : 0.f;
           uint4* dst = reinterpret_cast<uint4*>(
-              p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * kD + 64 * my_half);
+              p.out + (((size_t)q_base + i) * p.Hq + hq) * kD + 64 * my_half);
 #pragma unroll
           for (int c8 = 0; c8 < 8; ++c8) {
             uint32_t w[4];
@@ -792,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     const float inv = den > 0.f ? v_scale / den : 0.f;
     const int rr = row0 + r;
     const int i = rr / p.G, hq = h * p.G + rr % p.G;
-    __nv_bfloat16* dst = p.out + (((size_t)b * p.q_len + i) * p.Hq + hq) * kD + d0;
+    __nv_bfloat16* dst = p.out + (((size_t)q_base + i) * p.Hq + hq) * kD + d0;
     const __nv_bfloat162 lo = __floats2bfloat162_rn(o4.x * inv, o4.y * inv);
     const __nv_bfloat162 hi = __floats2bfloat162_rn(o4.z * inv, o4.w * inv);
     uint2 pk;

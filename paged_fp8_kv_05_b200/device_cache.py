@@ -19,12 +19,12 @@ class DeviceWorkload:
     """
 
     def __init__(self, w: Workload, device="cuda", fill=0x7F, min_split_tokens=256,
-                 fill_cache=True, max_batch=None):
+                 fill_cache=True, max_batch=None, max_q_len=None):
         self.w = w
         self.device = torch.device(device)
         self.pool = ak.KVPool(w.num_pages, w.page_size, w.num_kv_heads, w.head_dim,
                               w.k_scale, w.v_scale, max_batch=max_batch or max(w.batch, 1),
-                              max_q_len=w.q_len, num_q_heads=w.num_q_heads,
+                              max_q_len=max(max_q_len or 0, w.q_len), num_q_heads=w.num_q_heads,
                               max_seq_len=max(w.max_seq_len, w.q_len), device=self.device,
                               min_split_tokens=min_split_tokens, fill=fill)
         self.block_table = torch.from_numpy(np.ascontiguousarray(w.block_table)).to(self.device)

@@ -312,3 +312,36 @@ def make_verify_logits(*, batch, num_drafts, vocab, seed=0, dtype=torch.bfloat16
             drafts[b, a[b]] = (planted[b, a[b]] + 1 + rr.integers(0, vocab - 1)) % vocab
     logits = torch.from_numpy(x).to(dtype)
     return logits, drafts, dict(planted=planted, agree=a, second=second)
+
+
+def make_rope_inputs(*, batch, n_new, num_q_heads, num_kv_heads, head_dim, max_pos,
+                     rope_base=500000.0, seed=0):
+    """Synthetic QKV projection output of the new tokens and a rotary table.
+
+    ``qkv`` bf16 ``[B, n_new, Hq + 2 Hkv, D]``: N(0, 1) draws rounded to bf16
+    (query heads, then key heads, then value heads).  ``cos_sin`` float32
+    ``[max_pos, D]``: the cos (columns 0 .. D/2 - 1) and sin (the rest) of the
+    angles ``pos * rope_base ** (-2 i / D)`` -- the LLaMA-style frequency
+    schedule (rope_base 500000 as in LLaMA-3), evaluated in float64 and
+    rounded to float32; an input table, the same for both sides."""
+    (s_x,) = np.random.SeedSequence(seed).spawn(1)
+    x = np.random.default_rng(s_x).standard_normal(
+        (batch, n_new, num_q_heads + 2 * num_kv_heads, head_dim), dtype=np.float32)
+    qkv = torch.from_numpy(x).to(torch.bfloat16)
+    inv = float(rope_base) ** (-np.arange(head_dim // 2, dtype=np.float64) * 2.0 / head_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv[None, :]
+    cos_sin = np.concatenate([np.cos(ang), np.sin(ang)], axis=1).astype(np.float32)
+    return qkv, cos_sin
+
+
+def make_packed_queries(*, q_lens, num_q_heads, head_dim, seed=0):
+    """Packed bf16 queries for ragged verify / prefill: ``q`` ``[sum q_lens,
+    Hq, D]`` N(0, 1) rounded to bf16, and ``cu_q_lens`` int32 ``[B + 1]``
+    (exclusive prefix sums of ``q_lens``)."""
+    (s_q,) = np.random.SeedSequence(seed).spawn(1)
+    ql = np.asarray(q_lens, dtype=np.int64)
+    cu = np.zeros(len(ql) + 1, np.int32)
+    cu[1:] = np.cumsum(ql)
+    x = np.random.default_rng(s_q).standard_normal((int(cu[-1]), num_q_heads, head_dim),
+                                                    dtype=np.float32)
+    return torch.from_numpy(x).to(torch.bfloat16), cu

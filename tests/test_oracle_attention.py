@@ -235,3 +235,62 @@ def test_v_layout_dim_matches_token_major():
     for t in range(16):
         g[:, :, 0, :, paged.GROUP_POS[t]] = v[:, :, t, :]
     assert np.array_equal(attention.paged_gqa_decode(v_layout="grp16", **dict(c4, v_pages=g)), base4)
+
+
+def _varlen_case(rng, Hq, Hkv, D, ps, lens, qlens):
+    c = _rand_case(rng, len(lens), Hq, Hkv, D, ps, lens, 1)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = torch.randn(int(cu[-1]), Hq, D, generator=torch.Generator().manual_seed(int(rng.integers(1 << 30))))
+    q = q.to(torch.bfloat16).to(torch.float64).numpy()
+    del c["q"], c["q_len"]
+    return dict(c, q=q, cu_q_lens=cu)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,ps,lens,qlens", [
+    (4, 2, 8, 4, [7, 9, 3], [1, 5, 3]),
+    (8, 2, 64, 16, [40, 33, 64], [2, 1, 17]),      # a 17-row prefill chunk
+    (6, 3, 16, 8, [12, 8, 20, 5], [4, 0, 2, 5]),   # a sequence with no new rows
+])
+def test_varlen_matches_torch_sdpa_per_sequence(Hq, Hkv, D, ps, lens, qlens):
+    """Each sequence's rows against torch SDPA (float64, GQA by
+    repeat_interleave, boolean causal mask with that sequence's q_len)."""
+    rng = np.random.default_rng(sum(lens))
+    c = _varlen_case(rng, Hq, Hkv, D, ps, lens, qlens)
+    got = attention.paged_gqa_decode_varlen(**c)
+    cu = c["cu_q_lens"]
+    for b, L in enumerate(lens):
+        ql = qlens[b]
+        if ql == 0:
+            continue
+        one = dict(q=c["q"][cu[b]:cu[b + 1]][None], k_pages=c["k_pages"], v_pages=c["v_pages"],
+                   k_scale=c["k_scale"], v_scale=c["v_scale"], block_table=c["block_table"][b:b + 1],
+                   seq_lens=np.array([L], np.int32), q_len=ql, page_size=ps)
+        ref = _torch_reference(one, 1.0 / math.sqrt(D))[0]
+        assert np.max(np.abs(got[cu[b]:cu[b + 1]] - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_varlen_with_equal_lengths_is_the_uniform_path():
+    rng = np.random.default_rng(8)
+    c = _rand_case(rng, 3, 8, 2, 16, 4, [9, 12, 30], 3)
+    uni = attention.paged_gqa_decode(**c)
+    cu = np.arange(4, dtype=np.int32) * 3
+    var = attention.paged_gqa_decode_varlen(c["q"].reshape(9, 8, 16), cu, c["k_pages"],
+                                            c["v_pages"], c["k_scale"], c["v_scale"],
+                                            c["block_table"], c["seq_lens"], 4)
+    assert np.array_equal(var.reshape(3, 3, 8, 16), uni)
+
+
+def test_varlen_rows_ignore_later_drafts_and_empty_sequences_stay_nan():
+    rng = np.random.default_rng(9)
+    c = _varlen_case(rng, 4, 1, 8, 4, [10, 6], [4, 0])
+    base = attention.paged_gqa_decode_varlen(**c)
+    assert np.all(np.isnan(base[4:]))               # no rows of sequence 1 (empty)
+    L, ql = 10, 4
+    for i in range(ql - 1):
+        kp = c["k_pages"].copy()
+        for t in range(L - ql + i + 1, L):
+            page, slot = c["block_table"][0][t // 4], t % 4
+            kp[page, 0, slot, :] = 0x3C
+        got = attention.paged_gqa_decode_varlen(**dict(c, k_pages=kp))
+        assert np.array_equal(got[:i + 1], base[:i + 1])
+        assert not np.array_equal(got[i + 1:4], base[i + 1:4])
