@@ -250,6 +250,39 @@ ATLAS_API atlas_status_t atlas_rope_fp8_kv_append(const atlas_kv_pool_t* pool, c
                                                   int32_t n_new, void* q_out, void* stream);
 
 /*
+ * Finer-grained FP8 scales (Atlas deep-dive, ainews.cool, "Quantisation"
+ * paragraph: FP8 with per-group scale factors; here the finest group, one
+ * token's row of one KV head).  The same append as atlas_fp8_kv_append, but
+ * each new token's K row and V row of each KV head get their own dynamic scale
+ * s = fp32(max |x|) / fp32(448) (IEEE division; 1.0 for an all-zero row) and
+ * code = E4M3(fp32(x) / s); the scales are stored at [page][head][slot] of
+ * k_tok_scale / v_tok_scale (device float32 [num_pages][num_kv_heads]
+ * [page_size], caller-owned, 16-byte aligned), and v_scale_bound (device
+ * float32 [num_kv_heads], caller-owned, zero before the first append of the
+ * cache) is raised to the largest V scale appended per head.  The pool's
+ * per-head scales are not used.  Bit-exact with that definition.
+ */
+ATLAS_API atlas_status_t atlas_fp8_kv_append_tokscale(
+    const atlas_kv_pool_t* pool, const void* k_new, const void* v_new, int32_t dtype,
+    const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* start_pos,
+    int32_t batch, int32_t n_new, float* k_tok_scale, float* v_tok_scale, float* v_scale_bound,
+    void* stream);
+
+/*
+ * Decode / verify over a cache filled by atlas_fp8_kv_append_tokscale: K is
+ * dequantised with its per-token scales (applied to the scores), V with its
+ * per-token scales (applied to the probabilities, relative to v_scale_bound
+ * so that they stay in E4M3 range).  head_dim 128 only (the tensor-core
+ * kernel; ATLAS_ERR_UNSUPPORTED otherwise).  Uses the pool's pages; other
+ * arguments and errors as atlas_paged_gqa_decode.
+ */
+ATLAS_API atlas_status_t atlas_paged_gqa_decode_tokscale(
+    const atlas_kv_pool_t* pool, const void* q, const float* k_tok_scale,
+    const float* v_tok_scale, const float* v_scale_bound, const int32_t* block_table,
+    int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+    int32_t q_len, int32_t max_seq_len, float sm_scale, void* out, void* stream);
+
+/*
  * Paged decode (q_len == 1) / MTP-verify (q_len > 1) grouped-query attention.
  * q: device bf16 [batch][q_len][num_q_heads][head_dim], 16-byte aligned.
  * k_pages / v_pages: the pool's page arrays (or arrays of identical shape).

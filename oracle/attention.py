@@ -119,3 +119,35 @@ def paged_gqa_decode_varlen(q, cu_q_lens, k_pages, v_pages, k_scale, v_scale, bl
                 out[rows, hq, :] = attend(q[rows, hq, :], K[:, h, :], V[:, h, :], limits,
                                           sm_scale)
     return out
+
+
+def paged_gqa_decode_tokscale(q, k_pages, v_pages, k_tok_scale, v_tok_scale, block_table,
+                              seq_lens, q_len, page_size, sm_scale=None, sequences=None,
+                              k_layout="tok", v_layout="tok"):
+    """The same attention over a cache quantised with one dynamic scale per
+    (token, KV head) (``paged.append_tokscale``): K and V are dequantised with
+    the per-token scales ``[P, Hkv, ps]``, everything else as
+    :func:`paged_gqa_decode`."""
+    q = np.asarray(q, dtype=np.float64)
+    B, ql, Hq, D = q.shape
+    assert ql == q_len
+    Hkv = np.asarray(k_pages).shape[1]
+    G = Hq // Hkv
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / math.sqrt(D)
+    out = np.full((B, q_len, Hq, D), np.nan)
+    for b in (range(B) if sequences is None else sequences):
+        L = int(seq_lens[b])
+        if L < q_len:
+            raise ValueError(f"sequence {b}: seq_len {L} < q_len {q_len}")
+        K = paged.gather_dequant_tokscale(k_pages, k_tok_scale, block_table, b, L, page_size,
+                                          k_layout)
+        V = paged.gather_dequant_tokscale(v_pages, v_tok_scale, block_table, b, L, page_size,
+                                          v_layout)
+        limits = [L - q_len + i for i in range(q_len)]
+        for h in range(Hkv):
+            for g in range(G):
+                hq = h * G + g
+                out[b, :, hq, :] = attend(q[b, :, hq, :], K[:, h, :], V[:, h, :], limits,
+                                          sm_scale)
+    return out

@@ -91,3 +91,22 @@ def encode_value(y) -> np.ndarray:
 def encode(x, scale) -> np.ndarray:
     """Quantise ``x`` with ``scale``: ``encode_value(fp32(x) / fp32(scale))``."""
     return encode_value(quotient_f32(x, scale))
+
+
+def row_scale(x) -> np.ndarray:
+    """Dynamic per-row scale of the finer-grained reading (one scale per token
+    and KV head): ``fp32(max |x|) / fp32(448)`` over the last axis, as one
+    IEEE binary32 division; an all-zero row gets 1.0.  The Atlas deep-dive
+    (ainews.cool, "Quantisation" paragraph) names per-group scale factors; a
+    token's row of one head is the finest group."""
+    a = np.max(np.abs(np.asarray(x, dtype=np.float32)), axis=-1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s = np.divide(a, np.float32(MAX_FINITE), dtype=np.float32)
+    return np.where(a > 0, s, np.float32(1.0)).astype(np.float32)
+
+
+def encode_rows(x):
+    """(codes, scales): each row (last axis) of ``x`` quantised with its own
+    :func:`row_scale`."""
+    s = row_scale(x)
+    return encode(x, s[..., None]), s

@@ -127,3 +127,33 @@ def gather_dequant(pages, scale, block_table, b: int, length: int, page_size: in
     codes = gather_codes(pages, block_table, b, length, page_size, layout)
     scale = np.asarray(scale, dtype=np.float32).astype(np.float64)
     return e4m3.decode(codes) * scale[None, :, None]
+
+
+def append_tokscale(pages, scales, new, block_table, start_pos, page_size, layout="tok"):
+    """Finer-grained scales: like :func:`append`, but each new token's row of
+    each KV head is quantised with its own dynamic scale (``e4m3.row_scale``),
+    stored in ``scales`` float32 ``[P, Hkv, ps]`` at the token's (page, head,
+    slot).  Returns ``(pages', scales')``."""
+    out = np.array(pages, dtype=np.uint8, copy=True)
+    sc = np.array(scales, dtype=np.float32, copy=True)
+    new = np.asarray(new, dtype=np.float32)
+    B, n_new = new.shape[0], new.shape[1]
+    for b in range(B):
+        for t in range(n_new):
+            page, slot = slot_of(block_table, b, int(start_pos[b]) + t, page_size)
+            codes, s = e4m3.encode_rows(new[b, t])          # [Hkv, D], [Hkv]
+            _store(out, page, slot, codes, layout)
+            sc[page, :, slot] = s
+    return out, sc
+
+
+def gather_dequant_tokscale(pages, scales, block_table, b: int, length: int, page_size: int,
+                            layout="tok"):
+    """Dequantised float64 ``[length, Hkv, D]`` with per-token scales:
+    ``decode(code) * scales[page, h, slot]``."""
+    codes = gather_codes(pages, block_table, b, length, page_size, layout)
+    n_pages = (length + page_size - 1) // page_size
+    ids = np.asarray(block_table[b, :n_pages], dtype=np.int64)
+    s = np.asarray(scales, dtype=np.float32)[ids]                 # [n_pages, Hkv, ps]
+    s = s.transpose(0, 2, 1).reshape(n_pages * page_size, -1)[:length]
+    return e4m3.decode(codes) * s.astype(np.float64)[:, :, None]

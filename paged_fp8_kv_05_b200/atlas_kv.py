@@ -72,6 +72,12 @@ _SIGNATURES = [
       _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_plan", ctypes.c_int,
      [_c_ptr, _c_i32, _c_i32, _c_i32, _c_i32, ctypes.POINTER(_c_i32), _c_i32]),
+    ("atlas_fp8_kv_append_tokscale", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_ptr, _c_ptr,
+      _c_ptr, _c_ptr]),
+    ("atlas_paged_gqa_decode_tokscale", ctypes.c_int,
+     [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32, _c_i32, _c_i32,
+      _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
     ("atlas_paged_gqa_decode_varlen", ctypes.c_int,
      [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32, _c_ptr, _c_i32,
       _c_i32, _c_i32, _c_i32, ctypes.c_float, _c_ptr, _c_ptr]),
@@ -264,6 +270,50 @@ def atlas_paged_gqa_decode_noalloc(q, k_pages, v_pages, k_scale, v_scale, block_
                                                Hkv, D, ps, P, q_len, int(max_seq_len),
                                                float(sm_scale), _ptr(out), _stream(stream)),
            "atlas_paged_gqa_decode_noalloc")
+    return out
+
+
+class TokenScales:
+    """Per-(token, KV head) scale arrays of a pool in the finer-grained mode:
+    ``k``, ``v`` float32 ``[num_pages, num_kv_heads, page_size]`` and the
+    per-head V bound ``v_bound`` float32 ``[num_kv_heads]`` (zero-filled)."""
+
+    def __init__(self, pool: KVPool):
+        dev = pool.k_pages.device
+        shape = (pool.num_pages, pool.num_kv_heads, pool.page_size)
+        self.k = torch.zeros(shape, dtype=torch.float32, device=dev)
+        self.v = torch.zeros(shape, dtype=torch.float32, device=dev)
+        self.v_bound = torch.zeros(pool.num_kv_heads, dtype=torch.float32, device=dev)
+
+
+def atlas_fp8_kv_append_tokscale(pool: KVPool, scales: TokenScales, k_new, v_new, block_table,
+                                 start_pos, stream=None):
+    """Append with one dynamic scale per (token, KV head) into ``scales``."""
+    assert k_new.shape == v_new.shape and k_new.dtype == v_new.dtype
+    assert k_new.is_contiguous() and v_new.is_contiguous() and block_table.is_contiguous()
+    dtype = {torch.float32: ATLAS_DTYPE_F32, torch.bfloat16: ATLAS_DTYPE_BF16}[k_new.dtype]
+    B, n_new = int(k_new.shape[0]), int(k_new.shape[1])
+    _check(_lib.atlas_fp8_kv_append_tokscale(pool.handle, _ptr(k_new), _ptr(v_new), dtype,
+                                             _ptr(block_table), int(block_table.shape[1]),
+                                             _ptr(start_pos), B, n_new, _ptr(scales.k),
+                                             _ptr(scales.v), _ptr(scales.v_bound),
+                                             _stream(stream)),
+           "atlas_fp8_kv_append_tokscale")
+
+
+def atlas_paged_gqa_decode_tokscale(pool: KVPool, scales: TokenScales, q, block_table, seq_lens,
+                                    max_seq_len, out=None, sm_scale=0.0, stream=None):
+    """Decode / verify over a cache with per-(token, KV head) scales."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and block_table.is_contiguous()
+    B, q_len, Hq, D = (int(x) for x in q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.atlas_paged_gqa_decode_tokscale(pool.handle, _ptr(q), _ptr(scales.k),
+                                                _ptr(scales.v), _ptr(scales.v_bound),
+                                                _ptr(block_table), int(block_table.shape[1]),
+                                                _ptr(seq_lens), B, Hq, q_len, int(max_seq_len),
+                                                float(sm_scale), _ptr(out), _stream(stream)),
+           "atlas_paged_gqa_decode_tokscale")
     return out
 
 

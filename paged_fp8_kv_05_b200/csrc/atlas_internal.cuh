@@ -28,6 +28,12 @@ struct AppendParams {
   const int32_t* start_pos;   // [B]
   int32_t* err;               // device error word
   int batch, n_new, Hkv, D, ps, num_pages, max_blocks;
+  // finer-grained scales (nullptr: the per-head k_scale / v_scale): one
+  // dynamic scale per (token, KV head), [P][Hkv][ps], and the per-head bound
+  // of the V scales, [Hkv] (raised with atomicMax)
+  float* k_tok_scale;
+  float* v_tok_scale;
+  float* v_scale_bound;
 };
 
 struct DecodeParams {
@@ -63,6 +69,11 @@ struct DecodeParams {
   // issues the bulk copies of its unit number test_skip_unit, so the wait for
   // them runs out (no copy is in flight for that stage); -1 in normal use
   int test_skip_unit;
+  // finer-grained scales (tensor-core kernel only): per-(token, KV head) K and
+  // V scales [P][Hkv][ps]; then v_scale holds the heads' bounds of the V scales
+  // and k_scale is not read.  nullptr: the per-head scales.
+  const float* k_tok_scale;
+  const float* v_tok_scale;
 };
 
 constexpr unsigned long long kDefaultWaitLimitNs = 200ull * 1000 * 1000;
@@ -288,7 +299,7 @@ cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg,
 // (segment, split); stages 2 or 3.
 cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
                              cudaStream_t stream);
-size_t decode_tc_smem_bytes(int stages, int split_tokens);
+size_t decode_tc_smem_bytes(int stages, int split_tokens, bool tok_scales);
 
 // Dynamic shared memory of one decode CTA (rows = min(rows_per_cta, q_len * G)).
 size_t decode_fp8_smem_bytes(int D, int stages, int rbg, int rows, int max_units,

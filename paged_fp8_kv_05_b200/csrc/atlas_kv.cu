@@ -271,10 +271,11 @@ atlas_status_t atlas_kv_pool_set_option(atlas_kv_pool_t* pool, int32_t option, i
   return ATLAS_ERR_INVALID_ARG;
 }
 
-atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_new,
-                                   const void* v_new, int32_t dtype, const int32_t* block_table,
-                                   int32_t max_blocks_per_seq, const int32_t* start_pos,
-                                   int32_t batch, int32_t n_new, void* stream) {
+static atlas_status_t append_impl(const atlas_kv_pool_t* pool, const void* k_new,
+                                  const void* v_new, int32_t dtype, const int32_t* block_table,
+                                  int32_t max_blocks_per_seq, const int32_t* start_pos,
+                                  int32_t batch, int32_t n_new, float* k_tok_scale,
+                                  float* v_tok_scale, float* v_scale_bound, void* stream) {
   if (!pool) return ATLAS_ERR_INVALID_ARG;
   if (batch < 0 || n_new < 0 || max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
   if (dtype != ATLAS_DTYPE_F32 && dtype != ATLAS_DTYPE_BF16) return ATLAS_ERR_INVALID_ARG;
@@ -299,8 +300,31 @@ atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_ne
   p.ps = pool->page_size;
   p.num_pages = pool->num_pages;
   p.max_blocks = max_blocks_per_seq;
+  p.k_tok_scale = k_tok_scale;
+  p.v_tok_scale = v_tok_scale;
+  p.v_scale_bound = v_scale_bound;
   cudaError_t e = atlas::launch_fp8_append(p, device_sm_count(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+atlas_status_t atlas_fp8_kv_append(const atlas_kv_pool_t* pool, const void* k_new,
+                                   const void* v_new, int32_t dtype, const int32_t* block_table,
+                                   int32_t max_blocks_per_seq, const int32_t* start_pos,
+                                   int32_t batch, int32_t n_new, void* stream) {
+  return append_impl(pool, k_new, v_new, dtype, block_table, max_blocks_per_seq, start_pos,
+                     batch, n_new, nullptr, nullptr, nullptr, stream);
+}
+
+atlas_status_t atlas_fp8_kv_append_tokscale(const atlas_kv_pool_t* pool, const void* k_new,
+                                            const void* v_new, int32_t dtype,
+                                            const int32_t* block_table, int32_t max_blocks_per_seq,
+                                            const int32_t* start_pos, int32_t batch, int32_t n_new,
+                                            float* k_tok_scale, float* v_tok_scale,
+                                            float* v_scale_bound, void* stream) {
+  if (!k_tok_scale || !v_tok_scale || !v_scale_bound) return ATLAS_ERR_INVALID_ARG;
+  if (!aligned(k_tok_scale, 16) || !aligned(v_tok_scale, 16)) return ATLAS_ERR_INVALID_ARG;
+  return append_impl(pool, k_new, v_new, dtype, block_table, max_blocks_per_seq, start_pos,
+                     batch, n_new, k_tok_scale, v_tok_scale, v_scale_bound, stream);
 }
 
 atlas_status_t atlas_rope_fp8_kv_append(const atlas_kv_pool_t* pool, const void* qkv,
@@ -386,7 +410,9 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
                                   const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
                                   int32_t q_len, int32_t max_seq_len, float sm_scale, void* out,
                                   const void* k_new, const void* v_new, int32_t new_dtype,
-                                  void* stream, const int32_t* cu_q = nullptr) {
+                                  void* stream, const int32_t* cu_q = nullptr,
+                                  const float* k_tok_scale = nullptr,
+                                  const float* v_tok_scale = nullptr) {
   atlas_status_t st = check_decode_shape(pool, batch, num_q_heads, q_len, max_seq_len);
   if (st != ATLAS_OK) return st;
   if (max_blocks_per_seq < 1) return ATLAS_ERR_INVALID_ARG;
@@ -401,8 +427,15 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
 
   const int sms = device_sm_count();
   bool tc = false;
-  const atlas::DecodeLaunch L =
+  atlas::DecodeLaunch L =
       make_plan(pool, batch, num_q_heads, q_len, max_seq_len, sms, true, &tc, cu_q != nullptr);
+  if (k_tok_scale && !tc) {  // finer-grained scales: the tensor-core kernel only
+    if (pool->head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
+    tc = true;
+    L = atlas::plan_decode_tc(batch, num_q_heads, pool->num_kv_heads, q_len, max_seq_len, sms,
+                              pool->split_override, pool->stages_override,
+                              pool->waves_override > 0 ? pool->waves_override : 1);
+  }
   const WsLayout ws = ws_layout(L, pool->head_dim);
   if (ws.total > pool->workspace_bytes) return ATLAS_ERR_WORKSPACE;
   if (L.grid > 0x7FFFFFFFLL) return ATLAS_ERR_UNSUPPORTED;
@@ -445,6 +478,8 @@ static atlas_status_t decode_impl(const atlas_kv_pool_t* pool, const void* q,
   p.new_dtype = new_dtype;
   p.wait_limit_ns = pool->wait_limit_us > 0 ? 1000ull * pool->wait_limit_us
                                             : atlas::kDefaultWaitLimitNs;
+  p.k_tok_scale = k_tok_scale;
+  p.v_tok_scale = v_tok_scale;
   p.test_skip_unit = pool->test_skip_unit;
   cudaError_t e =
       tc ? atlas::launch_decode_tc(p, L.stages, L.grid, static_cast<cudaStream_t>(stream))
@@ -466,6 +501,27 @@ atlas_status_t atlas_paged_gqa_decode(const atlas_kv_pool_t* pool, const void* q
   return decode_impl(pool, q, k_pages, v_pages, k_scale, v_scale, block_table,
                      max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len, max_seq_len,
                      sm_scale, out, nullptr, nullptr, ATLAS_DTYPE_F32, stream);
+}
+
+atlas_status_t atlas_paged_gqa_decode_tokscale(const atlas_kv_pool_t* pool, const void* q,
+                                               const float* k_tok_scale,
+                                               const float* v_tok_scale,
+                                               const float* v_scale_bound,
+                                               const int32_t* block_table,
+                                               int32_t max_blocks_per_seq,
+                                               const int32_t* seq_lens, int32_t batch,
+                                               int32_t num_q_heads, int32_t q_len,
+                                               int32_t max_seq_len, float sm_scale, void* out,
+                                               void* stream) {
+  if (!pool) return ATLAS_ERR_INVALID_ARG;
+  if (pool->head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
+  if (batch > 0 && (!k_tok_scale || !v_tok_scale || !v_scale_bound)) return ATLAS_ERR_INVALID_ARG;
+  if (batch > 0 && (!aligned(k_tok_scale, 16) || !aligned(v_tok_scale, 16)))
+    return ATLAS_ERR_INVALID_ARG;
+  return decode_impl(pool, q, pool->k_pages, pool->v_pages, pool->k_scale, v_scale_bound,
+                     block_table, max_blocks_per_seq, seq_lens, batch, num_q_heads, q_len,
+                     max_seq_len, sm_scale, out, nullptr, nullptr, ATLAS_DTYPE_F32, stream,
+                     nullptr, k_tok_scale, v_tok_scale);
 }
 
 atlas_status_t atlas_paged_gqa_decode_varlen(const atlas_kv_pool_t* pool, const void* q,

@@ -223,13 +223,15 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // ----------------------------------------------------------- shared memory
 
 struct TcLayout {
-  size_t k, v, q, p, tab, bar, misc, rows, total;
+  size_t k, v, ts, q, p, tab, bar, misc, rows, total;
 };
-__host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces) {
+// ts: per-token K and V scales of each stage (finer-grained mode), else empty
+__host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool tok_scales) {
   TcLayout t;
   t.k = 0;                                              // [S][8 pieces][16 tok][128 B] (swizzled)
   t.v = t.k + (size_t)stages * kTileBytes;              // [S][8 pieces][128 d][16 slots]
-  t.q = t.v + (size_t)stages * kTileBytes;              // Q hi, Q lo: core-matrix layout
+  t.ts = t.v + (size_t)stages * kTileBytes;             // [S][K, V][128 tokens] float32
+  t.q = t.ts + (tok_scales ? (size_t)stages * 2 * kTile * 4 : 0);  // Q hi, Q lo: core matrices
   t.p = t.q + 2 * (size_t)kOpBytes;                     // P hi, P lo
   t.tab = t.p + 2 * (size_t)kOpBytes;                   // piece table, int32 per 16 tokens
   t.bar = (t.tab + (size_t)max_pieces * 4 + 15) / 16 * 16;
@@ -241,11 +243,17 @@ __host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int S>
+// TS: finer-grained scales -- one dynamic scale per (token, KV head) for K and
+// V (p.k_tok_scale / p.v_tok_scale, [P][Hkv][ps]), staged per tile beside the
+// codes; K scales multiply the scores, V scales (divided by the head's bound
+// p.v_scale[h], so that the probabilities stay in E4M3 range) the
+// probabilities of the PV product, and the bound scales the output.
+template <int S, bool TS>
 __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const TcLayout lay = tc_layout(S, p.split_tokens / 16);
+  const TcLayout lay = tc_layout(S, p.split_tokens / 16, TS);
+  float* sTS = reinterpret_cast<float*>(smem + lay.ts);  // [S][2][128]
   uint8_t* sK = smem + lay.k;
   uint8_t* sV = smem + lay.v;
   uint8_t* sQ = smem + lay.q;
@@ -307,7 +315,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   const bool whole = (n_parts == 1);
   const int row0 = rb * kRows;
   const int rows = min(kRows, Rtot - row0);
-  const float k_scale = __ldg(p.k_scale + h), v_scale = __ldg(p.v_scale + h);
+  // TS: the K scales are per token (applied to the scores) and p.v_scale[h] is
+  // the bound of the head's per-token V scales
+  const float k_scale = TS ? 1.f : __ldg(p.k_scale + h), v_scale = __ldg(p.v_scale + h);
 
   // ---- A0, fused append: the step's new tokens that fall in this split are
   // quantised and stored before any bulk copy reads the pages
@@ -460,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 #pragma unroll
         for (int pc = 0; pc < 8; ++pc) {
           const int k = 8 * j + pc;
-          if (k < n_pc && s_tab[k] >= 0) bytes += 2 * kPiece;
+          if (k < n_pc && s_tab[k] >= 0) bytes += 2 * kPiece + (TS ? 2 * 64 : 0);
         }
         if (bytes == 0) {
           mbar_arrive(&full_bar[st]);
@@ -477,6 +487,12 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
                     p.k_pages + (size_t)piece * kPiece, kPiece, &full_bar[st]);
           bulk_load(sV + (size_t)st * kTileBytes + pc * kPiece,
                     p.v_pages + (size_t)piece * kPiece, kPiece, &full_bar[st]);
+          if constexpr (TS) {  // the piece's 16 K and 16 V scales (64 bytes each)
+            bulk_load(sTS + (size_t)st * 2 * kTile + 16 * pc, p.k_tok_scale + (size_t)piece * 16,
+                      64, &full_bar[st]);
+            bulk_load(sTS + (size_t)st * 2 * kTile + kTile + 16 * pc,
+                      p.v_tok_scale + (size_t)piece * 16, 64, &full_bar[st]);
+          }
         }
       }
       if (*s_abort) {
@@ -584,6 +600,18 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) clean &= s_tab[(t0 - t_begin) / 16 + q4] >= 0;
       }
+      if constexpr (TS) {  // per-token K scales
+        const float4* ksc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile +
+                                                             64 * my_half);
+#pragma unroll
+        for (int k4 = 0; k4 < 16; ++k4) {
+          const float4 f = ksc[k4];
+          sv[4 * k4] = __float_as_uint(__uint_as_float(sv[4 * k4]) * f.x);
+          sv[4 * k4 + 1] = __float_as_uint(__uint_as_float(sv[4 * k4 + 1]) * f.y);
+          sv[4 * k4 + 2] = __float_as_uint(__uint_as_float(sv[4 * k4 + 2]) * f.z);
+          sv[4 * k4 + 3] = __float_as_uint(__uint_as_float(sv[4 * k4 + 3]) * f.w);
+        }
+      }
       if (clean) {
 #pragma unroll
         for (int k = 0; k < 64; ++k) x[k] = __uint_as_float(sv[k]) * row_scale2;
@@ -641,6 +669,21 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         lsum += pr[k];
       }
       l_run += lsum;
+      if constexpr (TS) {  // p * v_scale[t] / bound: at most p (masked tokens stay 0)
+        const float inv_bound = 1.f / v_scale;
+        const float4* vsc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile + kTile +
+                                                             64 * my_half);
+#pragma unroll
+        for (int k4 = 0; k4 < 16; ++k4) {
+          const float4 f = vsc[k4];
+          const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 4 * k4 + e;
+            pr[k] = pr[k] > 0.f ? pr[k] * (fv[e] * inv_bound) : 0.f;
+          }
+        }
+      }
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t hw[4], lw[4];
@@ -814,8 +857,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 
 }  // namespace
 
-size_t decode_tc_smem_bytes(int stages, int split_tokens) {
-  return tc_layout(stages, split_tokens / 16).total;
+size_t decode_tc_smem_bytes(int stages, int split_tokens, bool tok_scales) {
+  return tc_layout(stages, split_tokens / 16, tok_scales).total;
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
@@ -825,7 +868,8 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
   // at least 80 KB of shared memory per CTA: never more than two CTAs per SM,
   // so the two 256-column tensor-memory allocations always fit (an
   // allocation that cannot be served would wait)
-  size_t smem = decode_tc_smem_bytes(stages, p.split_tokens);
+  const bool ts = p.k_tok_scale != nullptr;
+  size_t smem = decode_tc_smem_bytes(stages, p.split_tokens, ts);
   if (smem < 80 * 1024) smem = 80 * 1024;
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -834,8 +878,8 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
     kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
   };
-  if (stages == 2) return go(paged_decode_tc_kernel<2>);
-  if (stages == 3) return go(paged_decode_tc_kernel<3>);
+  if (stages == 2) return ts ? go(paged_decode_tc_kernel<2, true>) : go(paged_decode_tc_kernel<2, false>);
+  if (stages == 3) return ts ? go(paged_decode_tc_kernel<3, true>) : go(paged_decode_tc_kernel<3, false>);
   return cudaErrorInvalidValue;
 }
 

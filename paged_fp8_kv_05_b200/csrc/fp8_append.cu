@@ -9,7 +9,12 @@
 // (cvt.rn.satfinite), sign of zero kept.  The result must be bit-exact with
 // that definition.
 //
-// Page layouts: K pages are token-major [P][Hkv][ps][D]; V pages are kept in
+// Finer-grained mode (k_tok_scale != nullptr): each token's row of each KV
+// head gets its own dynamic scale amax / 448, stored at [page][head][slot] of
+// the scale arrays, and the head's bound of the V scales is raised to it.
+//
+// Page layouts: K pages are token-major [P][Hkv][ps][D] (with D = 128 the
+// 16-byte chunk j of slot s sits at chunk position j XOR (s % 8)); V pages are kept in
 // groups of 16 slots, head-dim-major inside a group: [P][Hkv][ps/16][D][16]
 // (16 consecutive tokens of one head dimension adjacent), slot t of a group at
 // byte 4*((t%8)/2) + 2*(t/8) + t%2 (bytes 4c..4c+3 hold slots 2c, 2c+1, 2c+8,
@@ -30,7 +35,21 @@ namespace {
 
 constexpr int kTok = 16;  // tokens per CTA (one 16-slot V group when aligned)
 
-template <int D>
+// Dynamic per-(token, KV head) scale of the finer-grained mode: the largest
+// |x| over the token's D elements (held 16 per thread by the CH = D / 16
+// consecutive threads of the token), divided by 448 (IEEE division); 1 for an
+// all-zero row.  Every thread of the warp takes part in the shuffles.
+template <int CH>
+__device__ __forceinline__ float token_row_scale(const float (&x)[16]) {
+  float a = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) a = fmaxf(a, fabsf(x[k]));
+#pragma unroll
+  for (int o = 1; o < CH; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  return a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+}
+
+template <int D, bool TS>
 __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
   constexpr int CH = D / 16;  // 16-element chunks per row
   __shared__ __align__(16) uint8_t s_v[D][kTok];
@@ -62,17 +81,35 @@ __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
 
   const int pos = start + t0 + lt;
   const int page = s_page[lt];
-  if (lt < n_tok && page >= 0) {
-    const size_t src = (((size_t)b * p.n_new + t0 + lt) * p.Hkv + h) * D + 16 * j;
-    const size_t head_page = (size_t)page * p.Hkv + h;
-    float x[16];
+  const bool ok = lt < n_tok && page >= 0;
+  const size_t src = (((size_t)b * p.n_new + t0 + lt) * p.Hkv + h) * D + 16 * j;
+  const size_t head_page = ok ? (size_t)page * p.Hkv + h : 0;
+  const int slot = pos % p.ps;
+  float x[16];
+  if (ok) {
     load16_as_f32(p.k_new, src, p.dtype, x);
-    store16_k(p.k_pages, head_page, D, p.ps, pos % p.ps, j, quantize16_e4m3(x, __ldg(p.k_scale + h)));
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = 0.f;
+  }
+  const float ks = TS ? token_row_scale<D / 16>(x) : __ldg(p.k_scale + h);
+  if (ok) {
+    store16_k(p.k_pages, head_page, D, p.ps, slot, j, quantize16_e4m3(x, ks));
+    if (TS && j == 0) p.k_tok_scale[head_page * p.ps + slot] = ks;
     load16_as_f32(p.v_new, src, p.dtype, x);
-    const uint4 cv = quantize16_e4m3(x, __ldg(p.v_scale + h));
+  }
+  const float vs = TS ? token_row_scale<D / 16>(x) : __ldg(p.v_scale + h);
+  if (ok) {
+    const uint4 cv = quantize16_e4m3(x, vs);
     const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
     for (int k = 0; k < 16; ++k) s_v[16 * j + k][lt] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
+    if (TS && j == 0) {
+      p.v_tok_scale[head_page * p.ps + slot] = vs;
+      // positive floats order like their bit patterns: the head's running
+      // bound of the per-token V scales
+      atomicMax(reinterpret_cast<int*>(p.v_scale_bound + h), __float_as_int(vs));
+    }
   }
   __syncthreads();
 
@@ -113,10 +150,17 @@ cudaError_t launch_fp8_append(const AppendParams& p, int num_sms, cudaStream_t s
   const long long n_tiles = (p.n_new + kTok - 1) / kTok;
   const long long blocks = n_tiles * p.Hkv * p.batch;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  const bool ts = p.k_tok_scale != nullptr;
   if (p.D == 128) {
-    fp8_append_kernel<128><<<(unsigned)blocks, 128, 0, stream>>>(p);
+    if (ts)
+      fp8_append_kernel<128, true><<<(unsigned)blocks, 128, 0, stream>>>(p);
+    else
+      fp8_append_kernel<128, false><<<(unsigned)blocks, 128, 0, stream>>>(p);
   } else if (p.D == 64) {
-    fp8_append_kernel<64><<<(unsigned)blocks, 64, 0, stream>>>(p);
+    if (ts)
+      fp8_append_kernel<64, true><<<(unsigned)blocks, 64, 0, stream>>>(p);
+    else
+      fp8_append_kernel<64, false><<<(unsigned)blocks, 64, 0, stream>>>(p);
   } else {
     return cudaErrorInvalidValue;
   }

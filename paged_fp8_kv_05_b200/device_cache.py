@@ -19,7 +19,7 @@ class DeviceWorkload:
     """
 
     def __init__(self, w: Workload, device="cuda", fill=0x7F, min_split_tokens=256,
-                 fill_cache=True, max_batch=None, max_q_len=None):
+                 fill_cache=True, max_batch=None, max_q_len=None, token_scales=False):
         self.w = w
         self.device = torch.device(device)
         self.pool = ak.KVPool(w.num_pages, w.page_size, w.num_kv_heads, w.head_dim,
@@ -35,6 +35,8 @@ class DeviceWorkload:
             (w.seq_lens.astype(np.int64) - w.q_len).astype(np.int32)).to(self.device)
         self.k_new = torch.from_numpy(w.new_tokens("k")).to(self.device).contiguous()
         self.v_new = torch.from_numpy(w.new_tokens("v")).to(self.device).contiguous()
+        # finer-grained mode: one dynamic scale per (token, KV head)
+        self.scales = ak.TokenScales(self.pool) if token_scales else None
         if fill_cache:
             self.fill_prefix()
             self.append_new()
@@ -50,15 +52,28 @@ class DeviceWorkload:
                 continue
             kb = torch.from_numpy(w.seq_k(b)[:n]).to(self.device).unsqueeze(0).contiguous()
             vb = torch.from_numpy(w.seq_v(b)[:n]).to(self.device).unsqueeze(0).contiguous()
-            ak.atlas_fp8_kv_append(self.pool, kb, vb, self.block_table[b:b + 1], zero)
+            if self.scales is not None:
+                ak.atlas_fp8_kv_append_tokscale(self.pool, self.scales, kb, vb,
+                                                self.block_table[b:b + 1], zero)
+            else:
+                ak.atlas_fp8_kv_append(self.pool, kb, vb, self.block_table[b:b + 1], zero)
 
     def append_new(self, stream=None):
         """A0: quantise and scatter the step's q_len new tokens of every sequence."""
+        if self.scales is not None:
+            ak.atlas_fp8_kv_append_tokscale(self.pool, self.scales, self.k_new, self.v_new,
+                                            self.block_table, self.start_new, stream=stream)
+            return
         ak.atlas_fp8_kv_append(self.pool, self.k_new, self.v_new, self.block_table,
                                self.start_new, stream=stream)
 
     def decode(self, stream=None, out=None):
         """A1-A9: attention of the q_len new rows over the paged cache."""
+        if self.scales is not None:
+            return ak.atlas_paged_gqa_decode_tokscale(
+                self.pool, self.scales, self.q, self.block_table, self.seq_lens,
+                max(self.w.max_seq_len, self.w.q_len), out=self.out if out is None else out,
+                stream=stream)
         return ak.atlas_paged_gqa_decode(self.pool, self.q, self.block_table, self.seq_lens,
                                          max(self.w.max_seq_len, self.w.q_len),
                                          out=self.out if out is None else out, stream=stream)
