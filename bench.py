@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--kernel", type=int, default=0,
                     help="0 auto, 1 FP8 warp-MMA kernel, 2 tensor-core (tcgen05) kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the records of the rows after the core path")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -371,6 +373,115 @@ def append_throughput(w, device, flush_l2, ak, n_new=1024, calls=20):
             "launches_per_call": 1}
 
 
+def _time_calls(fn, flush_l2, device, calls=20, warm=3):
+    """Mean event-timed duration (ms) of fn() over `calls` calls, L2 flushed
+    before each (outside the events)."""
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warm):
+        fn()
+    times = []
+    for _ in range(calls):
+        flush_l2()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        z.record(stream)
+        z.synchronize()
+        times.append(a.elapsed_time(z))
+    return sum(times) / len(times)
+
+
+def next_rows(device, flush_l2, ak):
+    """The rows after the hot path's core: finer-grained scales (decode over a
+    per-token-scaled cache, LLaMA-3-8B decode shape), fused RoPE + FP8 append
+    (a 1024-token fill of that shape), ragged MTP verify (27B-class shape,
+    q_len 1..5 per sequence, batch 128) and a 512-row prefill chunk over 4096
+    tokens.  Each: one launch per call, event-timed with L2 flushed before
+    every call; bytes are the algorithmic bytes of the call."""
+    from paged_fp8_kv_05_b200 import workloads
+    from paged_fp8_kv_05_b200.device_cache import DeviceWorkload
+    peak, _ = load_peaks()
+    out = {}
+
+    def rec(what, ms, nbytes, extra=None):
+        r = {"what": what, "us_per_call": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+             "frac": nbytes / (ms * 1e-3) / 1e9 / peak, "bytes_per_call": nbytes,
+             "launches_per_call": 1}
+        if extra:
+            r.update(extra)
+        return r
+
+    # finer-grained scales: decode over a cache with one scale per (token, KV head)
+    w = workloads.config_workload(1)
+    dw = DeviceWorkload(w, device=device, token_scales=True)
+    b_dec, _ = algorithmic_bytes(w)
+    tok_bytes = b_dec + 2 * 4 * int(w.seq_lens.astype(np.int64).sum()) * w.num_kv_heads
+    ms = _time_calls(lambda: dw.decode(), flush_l2, device)
+    plain = DeviceWorkload(w, device=device)
+    ms_plain = _time_calls(lambda: plain.decode(), flush_l2, device)
+    out["token_scales"] = rec("atlas_paged_gqa_decode_tokscale, " + workloads.workload_tag(1),
+                              ms, tok_bytes, {"per_head_scales_us": ms_plain * 1e3,
+                                              "per_head_kernel": plain.plan()["kernel"]})
+    del dw, plain
+
+    # fused RoPE + quantise + append of a 1024-token fill, LLaMA-3-8B heads
+    B, n_new, Hq, Hkv, D, ps = 32, 1024, 32, 8, 128, 16
+    qkv, cos_sin = workloads.make_rope_inputs(batch=B, n_new=n_new, num_q_heads=Hq,
+                                              num_kv_heads=Hkv, head_dim=D, max_pos=n_new, seed=2)
+    pool = ak.KVPool(B * n_new // ps, ps, Hkv, D, np.full(Hkv, 0.01, np.float32),
+                     np.full(Hkv, 0.01, np.float32), max_batch=B, max_q_len=1, num_q_heads=Hq,
+                     max_seq_len=n_new, device=device)
+    table = torch.arange(B * n_new // ps, dtype=torch.int32, device=device).view(B, -1)
+    start = torch.zeros(B, dtype=torch.int32, device=device)
+    d_qkv, d_cs = qkv.to(device).contiguous(), torch.from_numpy(cos_sin).to(device)
+    q_out = torch.empty(B, n_new, Hq, D, dtype=torch.bfloat16, device=device)
+    ms = _time_calls(lambda: ak.atlas_rope_fp8_kv_append(pool, d_qkv, Hq, d_cs, table, start,
+                                                         q_out=q_out), flush_l2, device)
+    elems = B * n_new * (Hq + 2 * Hkv) * D
+    nbytes = elems * 2 + B * n_new * Hq * D * 2 + B * n_new * 2 * Hkv * D + B * n_new * D * 4
+    out["rope_append"] = rec(f"atlas_rope_fp8_kv_append, bf16 QKV {B} x {n_new} x "
+                             f"({Hq} + 2 x {Hkv}) x {D}", ms, nbytes)
+    del pool, d_qkv, q_out
+
+    # ragged MTP verify and a prefill chunk (packed rows)
+    for name, mk, qls in (
+            ("ragged_verify",
+             lambda: workloads.make_workload(batch=128, num_q_heads=40, num_kv_heads=8,
+                                             head_dim=128, page_size=16, q_len=1,
+                                             num_pages=16384, lengths=("uniform", 128, 1152),
+                                             seed=13),
+             lambda: np.random.default_rng(13).integers(1, 6, size=128)),
+            ("prefill_512_over_4096",
+             lambda: workloads.make_workload(batch=8, num_q_heads=32, num_kv_heads=8,
+                                             head_dim=128, page_size=16, q_len=1,
+                                             num_pages=8 * 256 + 8,
+                                             lengths=("fixed", [4096] * 8), seed=14),
+             lambda: np.full(8, 512))):
+        w = mk()
+        q_lens = qls()
+        q, cu = workloads.make_packed_queries(q_lens=q_lens, num_q_heads=w.num_q_heads,
+                                              head_dim=w.head_dim, seed=5)
+        dw = DeviceWorkload(w, device=device, max_q_len=int(q_lens.max()))
+        dq, dcu = q.to(device).contiguous(), torch.from_numpy(cu).to(device)
+        o = torch.empty_like(dq)
+        ms = _time_calls(lambda: ak.atlas_paged_gqa_decode_varlen(
+            dw.pool, dq, dcu, dw.block_table, dw.seq_lens, int(q_lens.max()), w.max_seq_len,
+            out=o), flush_l2, device)
+        L = w.seq_lens.astype(np.int64)
+        nbytes = (int(L.sum()) * w.num_kv_heads * w.head_dim * 2 + 2 * dq.numel() * 2
+                  + 4 * int(((L + 15) // 16).sum()))
+        flops = 4 * int(sum(int(L[b]) * int(q_lens[b]) for b in range(w.batch))) * w.num_q_heads * w.head_dim
+        out[name] = rec(f"atlas_paged_gqa_decode_varlen, {w.batch} sequences, q_len "
+                        f"{int(q_lens.min())}..{int(q_lens.max())}", ms, nbytes,
+                        {"tflops": flops / (ms * 1e-3) / 1e12,
+                         "plan": ak.atlas_paged_gqa_decode_plan(dw.pool, w.batch, w.num_q_heads,
+                                                                int(q_lens.max()),
+                                                                w.max_seq_len)})
+        del dw, dq, o
+    torch.cuda.empty_cache()
+    return out
+
+
 def accept_throughput(device, flush_l2, ak, batch=128, num_drafts=4, vocab=151936, calls=20):
     """Greedy MTP acceptance alone (the step after a verify decode): bf16
     verify logits [batch, K + 1, vocab] read once, plus the drafts in and the
@@ -573,6 +684,8 @@ def ours(args):
         "append": append_line,
         "accept": accept_throughput(device, flush_l2, ak),
     }
+    if not args.no_next_rows:
+        line["next_rows"] = next_rows(device, flush_l2, ak)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(head_w, args.cpu_seconds)
     if rank == 0:

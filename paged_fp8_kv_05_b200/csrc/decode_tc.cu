@@ -190,12 +190,17 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-// Two probabilities -> (hi, lo) E4M3 pairs: f16 rounding, hi = E4M3(x),
-// lo = E4M3(x - hi) (the subtraction is exact in f16).
-__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const uint32_t x = pack_f16x2(a, b);
-  hi = f16x2_to_e4m3x2(x);
-  lo = f16x2_to_e4m3x2(hsub2(x, e4m3x2_to_f16x2(hi)));
+// Two probabilities -> N E4M3 pairs: f16 rounding, then part k = E4M3 of what
+// the earlier parts leave (each subtraction is exact in f16).  Two parts
+// carry 8 significant bits, three carry the f16 value's 11.
+template <int N>
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t (&part)[N]) {
+  uint32_t x = pack_f16x2(a, b);
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    part[k] = f16x2_to_e4m3x2(x);
+    if (k + 1 < N) x = hsub2(x, e4m3x2_to_f16x2(part[k]));
+  }
 }
 
 // Byte of slot t inside a 16-slot V group row: bytes 4c..4c+3 hold slots
@@ -204,14 +209,28 @@ __device__ __forceinline__ int group_pos(int t) {
   return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
 }
 
+// One probe of an mbarrier phase without a suspend-time hint: the hand-offs
+// between the roles are short, and a thread put to sleep wakes up late.
+__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait that also gives up when another role has flagged an abort;
 // a wait that runs out raises the abort flag.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_probe(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_probe(bar, parity)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -225,6 +244,10 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 struct TcLayout {
   size_t k, v, ts, q, p, tab, bar, misc, rows, total;
 };
+// E4M3 parts that carry a probability into the PV product: hi + lo (8
+// significant bits); three with per-token V scales, where even the row's
+// largest probability is no longer a power of two
+__host__ __device__ constexpr int p_parts(bool tok_scales) { return tok_scales ? 3 : 2; }
 // ts: per-token K and V scales of each stage (finer-grained mode), else empty
 __host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool tok_scales) {
   TcLayout t;
@@ -233,9 +256,9 @@ __host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool t
   t.ts = t.v + (size_t)stages * kTileBytes;             // [S][K, V][128 tokens] float32
   t.q = t.ts + (tok_scales ? (size_t)stages * 2 * kTile * 4 : 0);  // Q hi, Q lo: core matrices
   t.p = t.q + 2 * (size_t)kOpBytes;                     // P hi, P lo
-  t.tab = t.p + 2 * (size_t)kOpBytes;                   // piece table, int32 per 16 tokens
+  t.tab = t.p + (size_t)p_parts(tok_scales) * kOpBytes; // piece table, int32 per 16 tokens
   t.bar = (t.tab + (size_t)max_pieces * 4 + 15) / 16 * 16;
-  t.misc = t.bar + (size_t)(2 * stages + 7) * 8;        // tmem address, abort flag, is_last
+  t.misc = t.bar + (size_t)(2 * stages + 8) * 8;        // tmem address, abort flag, is_last
   t.rows = t.misc + 16;                                 // merge: row reference, denominator
   t.total = t.rows + 2 * kRows * 4 + 1024;              // + slack for 1024-byte alignment
   return t;
@@ -267,6 +290,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   uint64_t* pfull_bar = bars + 2 * S + 4; // P written (and O rescaled)
   uint64_t* pvdone_bar = bars + 2 * S + 5;// PV of a tile done
   uint64_t* drain_bar = bars + 2 * S + 6; // every MMA of the CTA done
+  uint64_t* qready_bar = bars + 2 * S + 7; // Q written
+  constexpr int PARTS = p_parts(TS);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + lay.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + lay.misc + 4);
   int* s_is_last = reinterpret_cast<int*>(smem + lay.misc + 8);
@@ -366,70 +391,10 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     s_tab[k] = pc;
   }
 
-  // ---- Q rows as E4M3 hi + lo with a per-row power-of-two scale, in the
-  // K-major core-matrix layout of the A operand: row r, 16-dim chunk c at
-  // (r / 8) * 1024 + c * 128 + (r % 8) * 16
   const int my_row = 16 * (warp & 3) + (lane & 15);  // softmax warps: this thread's row
   const int my_half = lane >> 4;                     // tokens / dims 64 * half .. + 63
   float row_scale2 = 0.f;                            // score -> base-2 exponent
   int row_lim = -1;                                  // last visible key position
-  if (warp < 4) {
-    const int r = my_row, rr = row0 + r;
-    float x[64];
-    if (r < rows) {
-      const int i = rr / p.G, hq = h * p.G + rr % p.G;
-      const uint4* src = reinterpret_cast<const uint4*>(
-          p.q + (((size_t)q_base + i) * p.Hq + hq) * kD + 64 * my_half);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w = __ldg(src + c);
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          x[8 * c + 2 * k] = __uint_as_float(wv[k] << 16);
-          x[8 * c + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
-        }
-      }
-      row_lim = L - q_len + i;
-    } else {
-#pragma unroll
-      for (int k = 0; k < 64; ++k) x[k] = 0.f;
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 64; ++k) amax = fmaxf(amax, fabsf(x[k]));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 16));
-    // a = 2^(135 - e) puts amax in [256, 512); halve it if amax * a > 448
-    float a = 1.f;
-    if (amax > 0.f) {
-      const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF);
-      a = __uint_as_float((uint32_t)min(254, max(1, 262 - e)) << 23);
-      if (amax * a > 448.f) a *= 0.5f;
-    }
-    row_scale2 = k_scale * p.qk_scale_log2 / a;
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) {
-        const int k0 = 16 * cc + 4 * w4;
-        const float y0 = x[k0] * a, y1 = x[k0 + 1] * a, y2 = x[k0 + 2] * a, y3 = x[k0 + 3] * a;
-        const uint32_t h01 = f32x2_to_e4m3x2(y0, y1), h23 = f32x2_to_e4m3x2(y2, y3);
-        const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
-        const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
-        const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
-        const uint32_t l01 = f32x2_to_e4m3x2(y0 - b01.x, y1 - b01.y);
-        const uint32_t l23 = f32x2_to_e4m3x2(y2 - b23.x, y3 - b23.y);
-        hw[w4] = h01 | (h23 << 16);
-        lw[w4] = l01 | (l23 << 16);
-      }
-      const int off = (r >> 3) * 1024 + (4 * my_half + cc) * 128 + (r & 7) * 16;
-      *reinterpret_cast<uint4*>(sQ + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(sQ + kOpBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-    fence_proxy_async_shared();  // Q is read by the tensor core
-  }
-
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < S; ++s) {
@@ -443,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     mbar_init(pfull_bar, 128);
     mbar_init(pvdone_bar, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(qready_bar, 128);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -451,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     tmem_alloc(s_tmem, kTmemCols);
   }
   tc_fence_before();
-  __syncthreads();  // table, Q, barriers, tensor memory and appended tokens ready
+  __syncthreads();  // table, barriers, tensor memory and appended tokens ready
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint64_t limit = p.wait_limit_ns;
@@ -507,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       constexpr uint32_t idesc = idesc_f8(64, 64);
       const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = true;
+      bool ok = tc_wait(qready_bar, 0, s_abort, limit);
       auto pv = [&](int k) -> bool {  // O += P . V for tile k
         if (!tc_wait(pfull_bar, (uint32_t)(k & 1), s_abort, limit)) return false;
         tc_fence_after();
@@ -518,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         for (int dh = 0; dh < 2; ++dh) {
           const uint32_t d = tmem + ((uint32_t)(16 * dh) << 16) + kColO;
 #pragma unroll
-          for (int part = 0; part < 2; ++part)
+          for (int part = 0; part < PARTS; ++part)
             for (int ks = 0; ks < nks; ++ks) {
               const uint64_t a =
                   smem_desc(p_addr + part * kOpBytes + ks * 256, 128, 1024, 0);
@@ -566,6 +532,68 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // (first the Q rows, while the producer's first copies are in flight)
+  // ---- Q rows as E4M3 hi + lo with a per-row power-of-two scale, in the
+  // K-major core-matrix layout of the A operand: row r, 16-dim chunk c at
+  // (r / 8) * 1024 + c * 128 + (r % 8) * 16
+  {
+    const int r = my_row, rr = row0 + r;
+    float x[64];
+    if (r < rows) {
+      const int i = rr / p.G, hq = h * p.G + rr % p.G;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          p.q + (((size_t)q_base + i) * p.Hq + hq) * kD + 64 * my_half);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w = __ldg(src + c);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[8 * c + 2 * k] = __uint_as_float(wv[k] << 16);
+          x[8 * c + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
+        }
+      }
+      row_lim = L - q_len + i;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 64; ++k) x[k] = 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) amax = fmaxf(amax, fabsf(x[k]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 16));
+    // a = 2^(135 - e) puts amax in [256, 512); halve it if amax * a > 448
+    float a = 1.f;
+    if (amax > 0.f) {
+      const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+      a = __uint_as_float((uint32_t)min(254, max(1, 262 - e)) << 23);
+      if (amax * a > 448.f) a *= 0.5f;
+    }
+    row_scale2 = k_scale * p.qk_scale_log2 / a;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        const int k0 = 16 * cc + 4 * w4;
+        const float y0 = x[k0] * a, y1 = x[k0 + 1] * a, y2 = x[k0 + 2] * a, y3 = x[k0 + 3] * a;
+        const uint32_t h01 = f32x2_to_e4m3x2(y0, y1), h23 = f32x2_to_e4m3x2(y2, y3);
+        const uint32_t f01 = e4m3x2_to_f16x2(h01), f23 = e4m3x2_to_f16x2(h23);
+        const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
+        const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
+        const uint32_t l01 = f32x2_to_e4m3x2(y0 - b01.x, y1 - b01.y);
+        const uint32_t l23 = f32x2_to_e4m3x2(y2 - b23.x, y3 - b23.y);
+        hw[w4] = h01 | (h23 << 16);
+        lw[w4] = l01 | (l23 << 16);
+      }
+      const int off = (r >> 3) * 1024 + (4 * my_half + cc) * 128 + (r & 7) * 16;
+      *reinterpret_cast<uint4*>(sQ + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sQ + kOpBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    fence_proxy_async_shared();  // Q is read by the tensor core
+    mbar_arrive(qready_bar);
+  }
+
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     const bool row_ok = my_row < rows;
     float m_run = -INFINITY, l_run = 0.f;
@@ -638,14 +666,19 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         m_run = mx;
         l_run *= alpha;
       }
-      // P's buffer and O are free once the previous tile's PV is done
-      if (j > 0) {
+      // O (rescaled here) and P's buffer (written below) are free once the
+      // previous tile's PV is done; wait for it here only when a row of the
+      // warp must rescale its O, else after the exponentials, which then run
+      // while that PV is in flight
+      bool pv_done = (j == 0);
+      if (j > 0 && __any_sync(kFull, move)) {
         ok = tc_wait(pvdone_bar, (uint32_t)((j - 1) & 1), s_abort, limit);
         if (!__all_sync(kFull, ok)) {
           aborted = true;
           break;
         }
-        if (__any_sync(kFull, move)) {  // rescale the moved rows' O (A7)
+        pv_done = true;
+        {  // rescale the moved rows' O (A7)
           tc_fence_after();
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2) {
@@ -658,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           }
         }
       }
-      // p = 2^(x - m + 8) -> E4M3 hi + lo, in V's slot order inside each
+      // p = 2^(x - m + 8) -> E4M3 parts, in V's slot order inside each
       // 16-token chunk (word c = slots 2c, 2c+1, 2c+8, 2c+9)
       const float off = 8.f - ((m_run == -INFINITY) ? 0.f : m_run);
       float pr[64];
@@ -684,20 +717,31 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           }
         }
       }
+      uint32_t pw[PARTS][4][4];  // [part][16-token chunk][word]
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t hw[4], lw[4];
+      for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t h0, l0, h1, l1;
-          split_pair(pr[16 * cc + 2 * c4], pr[16 * cc + 2 * c4 + 1], h0, l0);
-          split_pair(pr[16 * cc + 2 * c4 + 8], pr[16 * cc + 2 * c4 + 9], h1, l1);
-          hw[c4] = h0 | (h1 << 16);
-          lw[c4] = l0 | (l1 << 16);
+          uint32_t a0[PARTS], a1[PARTS];
+          split_pair<PARTS>(pr[16 * cc + 2 * c4], pr[16 * cc + 2 * c4 + 1], a0);
+          split_pair<PARTS>(pr[16 * cc + 2 * c4 + 8], pr[16 * cc + 2 * c4 + 9], a1);
+#pragma unroll
+          for (int q = 0; q < PARTS; ++q) pw[q][cc][c4] = a0[q] | (a1[q] << 16);
         }
+      if (!pv_done) {
+        ok = tc_wait(pvdone_bar, (uint32_t)((j - 1) & 1), s_abort, limit);
+        if (!__all_sync(kFull, ok)) {
+          aborted = true;
+          break;
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
         const int offp = (my_row >> 3) * 1024 + (4 * my_half + cc) * 128 + (my_row & 7) * 16;
-        *reinterpret_cast<uint4*>(sP + offp) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sP + kOpBytes + offp) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+#pragma unroll
+        for (int q = 0; q < PARTS; ++q)
+          *reinterpret_cast<uint4*>(sP + q * kOpBytes + offp) =
+              make_uint4(pw[q][cc][0], pw[q][cc][1], pw[q][cc][2], pw[q][cc][3]);
       }
       // V slots that hold no valid token of this tile (past the split, bad
       // page) are zeroed, so that 0 * garbage never reaches O

@@ -20,14 +20,14 @@
 // byte 4*((t%8)/2) + 2*(t/8) + t%2 (bytes 4c..4c+3 hold slots 2c, 2c+1, 2c+8,
 // 2c+9, the token order of the decode kernel's P fragments).
 // Memory-bound: per element 4 (f32) or 2 (bf16) bytes read, 1 byte written.
-// A CTA owns 16 consecutive new tokens of one (sequence, KV head): D/16 x 16
-// threads, each with 16 consecutive elements of one token row of K and of V
-// (64 B or 32 B of coalesced input each).  K codes go out as one 16-byte store
-// per thread.  V codes are transposed through shared memory: when the 16
-// tokens fill one 16-slot group of a page exactly (the cache-fill case), every
-// thread stores whole 16-byte group rows; otherwise (the few tokens of a
-// decode step) each valid code is stored as one byte.  Index arithmetic is
-// 32-bit and done once per CTA.
+// A CTA owns 16 consecutive new tokens of one (sequence, KV head), D threads.
+// K: thread (token, chunk) quantises 16 consecutive elements of one token row
+// and stores them as one 16-byte write.  V: thread d takes head dimension d of
+// the 16 tokens (every load instruction reads one token row across the CTA,
+// coalesced), so the group row of dimension d -- 16 codes in the group's slot
+// order -- is formed in registers and leaves as one 16-byte write when the 16
+// tokens fill one 16-slot group of a page exactly (the cache-fill case); the
+// few tokens of a decode step are stored as single bytes.
 #include "atlas_internal.cuh"
 
 namespace atlas {
@@ -52,8 +52,9 @@ __device__ __forceinline__ float token_row_scale(const float (&x)[16]) {
 template <int D, bool TS>
 __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
   constexpr int CH = D / 16;  // 16-element chunks per row
-  __shared__ __align__(16) uint8_t s_v[D][kTok];
+  constexpr int NW = D / 32;  // warps
   __shared__ int s_page[kTok];
+  __shared__ float s_amax[NW][kTok];
   const int n_tiles = (p.n_new + kTok - 1) / kTok;
   const int tile = blockIdx.x % n_tiles;
   const int bh = blockIdx.x / n_tiles;
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
   const int n_tok = min(kTok, p.n_new - t0);
   const int start = __ldg(p.start_pos + b);
   const int tid = threadIdx.x;
-  const int lt = tid / CH, j = tid % CH;  // token within the tile, chunk
+  const int lt = tid / CH, j = tid % CH;  // K: token within the tile, chunk
 
   if (tid < kTok) {  // page of each token of the tile (-1: not written, flagged)
     int page = -1;
@@ -77,68 +78,112 @@ __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
     }
     s_page[tid] = page;
   }
-  __syncthreads();
 
-  const int pos = start + t0 + lt;
-  const int page = s_page[lt];
-  const bool ok = lt < n_tok && page >= 0;
-  const size_t src = (((size_t)b * p.n_new + t0 + lt) * p.Hkv + h) * D + 16 * j;
-  const size_t head_page = ok ? (size_t)page * p.Hkv + h : 0;
-  const int slot = pos % p.ps;
-  float x[16];
-  if (ok) {
-    load16_as_f32(p.k_new, src, p.dtype, x);
-  } else {
+  // ---- V, one head dimension per thread: element d of the tile's 16 tokens
+  // (each load instruction reads one token's row across the CTA: coalesced),
+  // quantised and packed in the 16-slot group order -- one 16-byte store per
+  // thread when the tile is exactly one group of one page
+  const int d = tid;
+  float xv[kTok];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) x[k] = 0.f;
-  }
-  const float ks = TS ? token_row_scale<D / 16>(x) : __ldg(p.k_scale + h);
-  if (ok) {
-    store16_k(p.k_pages, head_page, D, p.ps, slot, j, quantize16_e4m3(x, ks));
-    if (TS && j == 0) p.k_tok_scale[head_page * p.ps + slot] = ks;
-    load16_as_f32(p.v_new, src, p.dtype, x);
-  }
-  const float vs = TS ? token_row_scale<D / 16>(x) : __ldg(p.v_scale + h);
-  if (ok) {
-    const uint4 cv = quantize16_e4m3(x, vs);
-    const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-    for (int k = 0; k < 16; ++k) s_v[16 * j + k][lt] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
-    if (TS && j == 0) {
-      p.v_tok_scale[head_page * p.ps + slot] = vs;
-      // positive floats order like their bit patterns: the head's running
-      // bound of the per-token V scales
-      atomicMax(reinterpret_cast<int*>(p.v_scale_bound + h), __float_as_int(vs));
+  for (int t = 0; t < kTok; ++t) {
+    xv[t] = 0.f;
+    if (t < n_tok) {
+      const size_t e = (((size_t)b * p.n_new + t0 + t) * p.Hkv + h) * D + d;
+      xv[t] = (p.dtype == ATLAS_DTYPE_F32)
+                  ? __ldg(static_cast<const float*>(p.v_new) + e)
+                  : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p.v_new) + e));
     }
   }
-  __syncthreads();
-
-  // V: slot t of a 16-slot group sits at byte 4*((t%8)/2) + 2*(t/8) + t%2 of
-  // the group row of each head dimension
-  const int p0 = start + t0;
-  const bool whole_group = n_tok == kTok && (p0 % 16) == 0 && s_page[0] >= 0;
-  if (whole_group) {  // thread d writes row d of the group (16 bytes)
-    const int d = tid;
-    uint32_t word[4] = {0u, 0u, 0u, 0u};
+  float vsc[kTok];
+  if constexpr (TS) {  // per-token scales: the row maximum over all D threads
 #pragma unroll
     for (int t = 0; t < kTok; ++t) {
-      const int byte = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
-      word[byte >> 2] |= (uint32_t)s_v[d][t] << (8 * (byte & 3));
+      float a = fabsf(xv[t]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      if ((tid & 31) == 0) s_amax[tid >> 5][t] = a;
     }
+  }
+  __syncthreads();  // s_page (and s_amax) ready
+  if constexpr (TS) {
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) {
+      float a = s_amax[0][t];
+#pragma unroll
+      for (int w = 1; w < NW; ++w) a = fmaxf(a, s_amax[w][t]);
+      vsc[t] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    }
+  } else {
+    const float s0 = __ldg(p.v_scale + h);
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) vsc[t] = s0;
+  }
+  uint32_t code[kTok];
+#pragma unroll
+  for (int t = 0; t < kTok; t += 2) {
+    const float y0 = __fdiv_rn(xv[t], vsc[t]), y1 = __fdiv_rn(xv[t + 1], vsc[t + 1]);
+    const uint32_t pr = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+    code[t] = pr & 0xFFu;
+    code[t + 1] = (pr >> 8) & 0xFFu;
+  }
+  const int p0 = start + t0;
+  const bool whole_group = n_tok == kTok && (p0 % 16) == 0 && s_page[0] >= 0;
+  if (whole_group) {
+    // slot t of the group sits at byte 4*((t%8)/2) + 2*(t/8) + t%2: word c
+    // holds slots 2c, 2c+1, 2c+8, 2c+9
+    uint32_t w[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      w[c] = code[2 * c] | (code[2 * c + 1] << 8) | (code[2 * c + 8] << 16) |
+             (code[2 * c + 9] << 24);
     const size_t head_page = (size_t)s_page[0] * p.Hkv + h;
     uint8_t* dst = p.v_pages + (head_page * (p.ps / 16) + (p0 % p.ps) / 16) * (16 * D) + 16 * d;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(word[0], word[1], word[2], word[3]);
-  } else {  // byte stores for the valid tokens
-    for (int idx = tid; idx < n_tok * D; idx += D) {
-      const int t = idx / D, d = idx % D;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {  // byte stores for the valid tokens (a decode step's few tokens)
+#pragma unroll
+    for (int t = 0; t < kTok; ++t) {
       const int pg = s_page[t];
-      if (pg < 0) continue;
+      if (t >= n_tok || pg < 0) continue;
       const int slot = (p0 + t) % p.ps;
       const int g = slot % 16;
       const int byte = 4 * ((g & 7) >> 1) + 2 * (g >> 3) + (g & 1);
       const size_t head_page = (size_t)pg * p.Hkv + h;
-      p.v_pages[(head_page * (p.ps / 16) + slot / 16) * (16 * D) + 16 * d + byte] = s_v[d][t];
+      p.v_pages[(head_page * (p.ps / 16) + slot / 16) * (16 * D) + 16 * d + byte] =
+          (uint8_t)code[t];
     }
+  }
+  if (TS && d < n_tok && s_page[d] >= 0) {  // thread t < 16 stores token t's V scale
+    float a = s_amax[0][d];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) a = fmaxf(a, s_amax[w][d]);
+    const float sc = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    const int slot = (p0 + d) % p.ps;
+    p.v_tok_scale[((size_t)s_page[d] * p.Hkv + h) * p.ps + slot] = sc;
+    // positive floats order like their bit patterns: the head's running bound
+    // of the per-token V scales
+    atomicMax(reinterpret_cast<int*>(p.v_scale_bound + h), __float_as_int(sc));
+  }
+
+  // ---- K, 16 consecutive elements of one token row per thread (one
+  // 16-byte store of codes each)
+  const int pos = start + t0 + lt;
+  const int page = s_page[lt];
+  const bool ok = lt < n_tok && page >= 0;
+  float x[16];
+  if (ok) {
+    load16_as_f32(p.k_new, (((size_t)b * p.n_new + t0 + lt) * p.Hkv + h) * D + 16 * j, p.dtype,
+                  x);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[k] = 0.f;
+  }
+  const float ks = TS ? token_row_scale<CH>(x) : __ldg(p.k_scale + h);
+  if (ok) {
+    const size_t head_page = (size_t)page * p.Hkv + h;
+    const int slot = pos % p.ps;
+    store16_k(p.k_pages, head_page, D, p.ps, slot, j, quantize16_e4m3(x, ks));
+    if (TS && j == 0) p.k_tok_scale[head_page * p.ps + slot] = ks;
   }
 }
 

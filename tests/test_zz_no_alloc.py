@@ -57,6 +57,9 @@ def test_noalloc_matches_pool_entry_point_on_two_calls(name):
     from paged_fp8_kv_05_b200.device_cache import DeviceWorkload
 
     dw = DeviceWorkload(w)
+    # the no-allocation entry point runs the FP8 warp-MMA kernel with the
+    # automatic partition; compare with the pool entry point on that kernel
+    dw.pool.set_option(ak.OPT_KERNEL, ak.KERNEL_WARP_MMA)
     ref = dw.decode(out=torch.empty_like(dw.q)).float()
     assert dw.pool.device_error() == 0
     needs = _partial_bytes(dw.plan(), w)
