@@ -94,3 +94,22 @@ def test_rope_append_flags_positions_outside_the_table(ak):
     k = pool.k_pages.cpu().numpy()
     assert np.all(k[4, :, 10:12] == 0x7F)          # rows 10, 11 of sequence 1 not written
     assert not np.all(k[4, :, 9] == 0x7F)
+
+
+def test_rope_append_aligned_window_crossing_the_table_end(ak):
+    """A full 16-token window starting at a group boundary whose last tokens
+    lie past the rotary table: those tokens' K and V rows stay unwritten (the
+    whole-row V store is not taken)."""
+    Hq, Hkv, D, ps = 4, 2, 128, 16
+    qkv, cos_sin = workloads.make_rope_inputs(batch=1, n_new=16, num_q_heads=Hq,
+                                              num_kv_heads=Hkv, head_dim=D, max_pos=10, seed=3)
+    pool = ak.KVPool(2, ps, Hkv, D, [0.01, 0.01], [0.01, 0.01], max_batch=1, max_q_len=1,
+                     num_q_heads=Hq, max_seq_len=32, fill=0x7F)
+    bt = torch.tensor([[1, 0]], dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ak.atlas_rope_fp8_kv_append(pool, qkv.cuda(), Hq, torch.from_numpy(cos_sin).cuda(), bt, st)
+    assert pool.device_error() & ak.DEVERR_APPEND
+    v = v_token_major(pool.v_pages.cpu().numpy())
+    k = pool.k_pages.cpu().numpy()
+    assert np.all(v[1, :, 10:16] == 0x7F) and np.all(k[1, :, 10:16] == 0x7F)
+    assert not np.all(v[1, :, 0:10] == 0x7F)
