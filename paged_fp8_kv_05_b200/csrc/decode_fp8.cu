@@ -733,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2)
 #pragma unroll 1
   for (int pi = 0; pi < n_port; ++pi) {
     const Portion P = s_port[pi];
-    const int b = P.b, seg = P.seg, L = P.L;
+    const int seg = P.seg, L = P.L;
     const int h = seg / RB, rg = seg % RB;
     const int Rtot = P.ql * p.G;           // this sequence's query rows per KV head
     const int cta_row0 = rg * RC;
