@@ -15,9 +15,10 @@
 // CTA = one split of one segment (sequence b, KV head h, block of up to 64
 // query rows), as in the grid partition: split_tokens KV tokens in tiles of
 // 128.  Six warps:
-//   * warp 4, lane 0 -- producer: 1-D bulk copies (cp.async.bulk, no
-//     multicast) of the tile's eight 16-token K pieces and eight V pieces into
-//     a ring of S stages, completion on a "full" mbarrier;
+//   * warp 4 -- producer: 1-D bulk copies (cp.async.bulk, no multicast) of
+//     the tile's eight 16-token K pieces and eight V pieces (pieces adjacent
+//     in a page go as one copy, one lane per run) into a ring of S stages,
+//     completion on a "full" mbarrier;
 //   * warp 5, lane 0 -- MMA issuer: per tile
 //       S[64 rows x 128 tok] = (Qhi + Qlo)[64 x 128 d] . K_tile^T
 //     as two M=64, N=64 halves (tokens 0-63 into TMEM lanes 0-15 of each warp
@@ -424,48 +425,57 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % S;
-        if (j >= S && !tc_wait(&empty_bar[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit))
-          break;
-        issued = j + 1;
-        if (p.test_skip_unit == j && cid == 0) continue;  // lost copy (tests only)
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int pc = 0; pc < 8; ++pc) {
-          const int k = 8 * j + pc;
-          if (k < n_pc && s_tab[k] >= 0) bytes += 2 * kPiece + (TS ? 2 * 64 : 0);
-        }
-        if (bytes == 0) {
+    // The whole warp: lane 0 waits for the stage and posts the byte count,
+    // then lanes 0-7 (K) and 8-15 (V) each issue the copy of one run of
+    // pieces that lie back to back in the page arrays (a page of 64 slots is
+    // four adjacent pieces), so the tile's copies go out in one instruction.
+    // A token-scale copy (64 bytes per piece) goes with every piece.
+    int issued = 0;
+    const int pc_l = lane & 7;
+    const bool is_v_lane = (lane & 8) != 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % S;
+      bool ok = true;
+      if (j >= S && lane == 0)
+        ok = tc_wait(&empty_bar[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
+      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      issued = j + 1;
+      if (p.test_skip_unit == j && cid == 0) continue;  // lost copy (tests only)
+      // this lane's piece and the run of adjacent pieces it starts
+      const int k = 8 * j + pc_l;
+      const int piece = (k < n_pc) ? s_tab[k] : -1;
+      const int prev = (pc_l > 0 && k - 1 < n_pc) ? s_tab[k - 1] : -2;
+      const bool starts = piece >= 0 && !(pc_l > 0 && prev >= 0 && prev + 1 == piece);
+      int run = 0;
+      if (starts) {
+        run = 1;
+        while (pc_l + run < 8 && k + run < n_pc && s_tab[k + run] == piece + run) ++run;
+      }
+      unsigned valid_mask = __ballot_sync(kFull, piece >= 0 && lane < 8);
+      const uint32_t bytes = (uint32_t)__popc(valid_mask) * (2 * kPiece + (TS ? 2 * 64 : 0));
+      if (lane == 0) {
+        if (bytes == 0)
           mbar_arrive(&full_bar[st]);
-          continue;
-        }
-        mbar_arrive_expect_tx(&full_bar[st], bytes);
-#pragma unroll 1
-        for (int pc = 0; pc < 8; ++pc) {
-          const int k = 8 * j + pc;
-          if (k >= n_pc) break;
-          const int piece = s_tab[k];
-          if (piece < 0) continue;
-          bulk_load(sK + (size_t)st * kTileBytes + pc * kPiece,
-                    p.k_pages + (size_t)piece * kPiece, kPiece, &full_bar[st]);
-          bulk_load(sV + (size_t)st * kTileBytes + pc * kPiece,
-                    p.v_pages + (size_t)piece * kPiece, kPiece, &full_bar[st]);
-          if constexpr (TS) {  // the piece's 16 K and 16 V scales (64 bytes each)
-            bulk_load(sTS + (size_t)st * 2 * kTile + 16 * pc, p.k_tok_scale + (size_t)piece * 16,
-                      64, &full_bar[st]);
-            bulk_load(sTS + (size_t)st * 2 * kTile + kTile + 16 * pc,
-                      p.v_tok_scale + (size_t)piece * 16, 64, &full_bar[st]);
-          }
+        else
+          mbar_arrive_expect_tx(&full_bar[st], bytes);
+      }
+      __syncwarp();
+      if (bytes != 0 && lane < 16 && starts) {
+        uint8_t* dst = (is_v_lane ? sV : sK) + (size_t)st * kTileBytes + pc_l * kPiece;
+        const uint8_t* src = (is_v_lane ? p.v_pages : p.k_pages) + (size_t)piece * kPiece;
+        bulk_load(dst, src, (uint32_t)run * kPiece, &full_bar[st]);
+        if constexpr (TS) {  // the run's K or V scales (64 bytes per piece)
+          bulk_load(sTS + (size_t)st * 2 * kTile + (is_v_lane ? kTile : 0) + 16 * pc_l,
+                    (is_v_lane ? p.v_tok_scale : p.k_tok_scale) + (size_t)piece * 16,
+                    (uint32_t)run * 64, &full_bar[st]);
         }
       }
-      if (*s_abort) {
-        // drain: copies of the last stages issued may still be in flight
-        for (int j = max(0, issued - S); j < issued; ++j)
-          mbar_wait_bounded(&full_bar[j % S], (uint32_t)((j / S) & 1), limit);
-      }
+    }
+    if (*s_abort && lane == 0) {
+      // drain: copies of the last stages issued may still be in flight
+      for (int j = max(0, issued - S); j < issued; ++j)
+        mbar_wait_bounded(&full_bar[j % S], (uint32_t)((j / S) & 1), limit);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
@@ -474,9 +484,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       bool ok = tc_wait(qready_bar, 0, s_abort, limit);
-      auto pv = [&](int k) -> bool {  // O += P . V for tile k
-        if (!tc_wait(pfull_bar, (uint32_t)(k & 1), s_abort, limit)) return false;
-        tc_fence_after();
+      auto issue_pv = [&](int k) {  // O += P . V for tile k
         const int st = k % S;
         const int tok = t_end - (t_begin + kTile * k);  // valid tokens of the tile (>= 1)
         const int nks = min(4, (tok + 31) / 32);       // 32-token k-steps holding any
@@ -495,19 +503,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         }
         mma_commit(&empty_bar[st]);
         mma_commit(pvdone_bar);
-        return true;
       };
-      for (int j = 0; j < n_tiles && ok; ++j) {
+      auto issue_s = [&](int j) {  // S = (Qhi + Qlo) . K^T for tile j
         const int st = j % S, sb = j & 1;
-        if (!tc_wait(&full_bar[st], (uint32_t)((j / S) & 1), s_abort, limit)) {
-          ok = false;
-          break;
-        }
-        if (j >= 2 && !tc_wait(&sfree_bar[sb], (uint32_t)(((j >> 1) - 1) & 1), s_abort, limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (t_begin + kTile * j + 64 * half >= t_end) break;  // no token in this half
@@ -523,9 +521,39 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
             }
         }
         mma_commit(&sfull_bar[sb]);
-        if (j >= 1 && !pv(j - 1)) ok = false;
+      };
+      // Event loop: S(js) once tile js has landed and its S buffer is free
+      // (at most two S tiles ahead of the PV products), PV(jp) once the
+      // softmax has written P(jp) -- whichever is ready first, so that a PV
+      // never waits behind the next tile's copies.  Bounded: no progress for
+      // the wait limit raises the abort flag.
+      int js = 0, jp = 0;
+      uint64_t t_idle = global_timer_ns();
+      while (ok && jp < n_tiles) {
+        bool progressed = false;
+        if (js < n_tiles && js < jp + 2 &&
+            mbar_probe(&full_bar[js % S], (uint32_t)((js / S) & 1)) &&
+            (js < 2 || mbar_probe(&sfree_bar[js & 1], (uint32_t)(((js >> 1) - 1) & 1)))) {
+          tc_fence_after();
+          issue_s(js);
+          ++js;
+          progressed = true;
+        }
+        if (jp < js && mbar_probe(pfull_bar, (uint32_t)(jp & 1))) {
+          tc_fence_after();
+          issue_pv(jp);
+          ++jp;
+          progressed = true;
+        }
+        if (progressed) {
+          t_idle = global_timer_ns();
+        } else if (*s_abort) {
+          ok = false;
+        } else if (global_timer_ns() - t_idle > limit) {
+          *s_abort = 1;
+          ok = false;
+        }
       }
-      if (ok) pv(n_tiles - 1);
       // every MMA issued so far has completed before tensor memory is released
       mma_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, limit);
@@ -655,9 +683,16 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 
       // online softmax (A6): the row's reference moves only when a score
       // exceeds it by more than 0.5; both threads of the row decide alike
-      float mx = -INFINITY;
+      float mx;
+      {  // eight independent chains, then a tree
+        float m8[8];
 #pragma unroll
-      for (int k = 0; k < 64; ++k) mx = fmaxf(mx, x[k]);
+        for (int e = 0; e < 8; ++e) m8[e] = x[e];
+#pragma unroll
+        for (int k = 8; k < 64; ++k) m8[k & 7] = fmaxf(m8[k & 7], x[k]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
       const bool move = mx > m_run + 0.5f;
       float alpha = 1.f;
@@ -695,13 +730,13 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       // 16-token chunk (word c = slots 2c, 2c+1, 2c+8, 2c+9)
       const float off = 8.f - ((m_run == -INFINITY) ? 0.f : m_run);
       float pr[64];
-      float lsum = 0.f;
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 64; ++k) {
         pr[k] = fast_exp2(x[k] + off);
-        lsum += pr[k];
+        ls8[k & 7] += pr[k];
       }
-      l_run += lsum;
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       if constexpr (TS) {  // p * v_scale[t] / bound: at most p (masked tokens stay 0)
         const float inv_bound = 1.f / v_scale;
         const float4* vsc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile + kTile +
