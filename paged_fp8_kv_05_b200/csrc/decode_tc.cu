@@ -224,6 +224,20 @@ __device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase (for the MMA issuer's event loop,
+// which polls two conditions and must not be parked on either).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait that also gives up when another role has flagged an abort;
 // a wait that runs out raises the abort flag.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -532,14 +546,14 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       while (ok && jp < n_tiles) {
         bool progressed = false;
         if (js < n_tiles && js < jp + 2 &&
-            mbar_probe(&full_bar[js % S], (uint32_t)((js / S) & 1)) &&
-            (js < 2 || mbar_probe(&sfree_bar[js & 1], (uint32_t)(((js >> 1) - 1) & 1)))) {
+            mbar_test(&full_bar[js % S], (uint32_t)((js / S) & 1)) &&
+            (js < 2 || mbar_test(&sfree_bar[js & 1], (uint32_t)(((js >> 1) - 1) & 1)))) {
           tc_fence_after();
           issue_s(js);
           ++js;
           progressed = true;
         }
-        if (jp < js && mbar_probe(pfull_bar, (uint32_t)(jp & 1))) {
+        if (jp < js && mbar_test(pfull_bar, (uint32_t)(jp & 1))) {
           tc_fence_after();
           issue_pv(jp);
           ++jp;
@@ -552,6 +566,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         } else if (global_timer_ns() - t_idle > limit) {
           *s_abort = 1;
           ok = false;
+        } else {
+          __nanosleep(32);  // leave issue slots to the softmax warp of this SM quarter
         }
       }
       // every MMA issued so far has completed before tensor memory is released
@@ -701,31 +717,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         m_run = mx;
         l_run *= alpha;
       }
-      // O (rescaled here) and P's buffer (written below) are free once the
-      // previous tile's PV is done; wait for it here only when a row of the
-      // warp must rescale its O, else after the exponentials, which then run
-      // while that PV is in flight
-      bool pv_done = (j == 0);
-      if (j > 0 && __any_sync(kFull, move)) {
-        ok = tc_wait(pvdone_bar, (uint32_t)((j - 1) & 1), s_abort, limit);
-        if (!__all_sync(kFull, ok)) {
-          aborted = true;
-          break;
-        }
-        pv_done = true;
-        {  // rescale the moved rows' O (A7)
-          tc_fence_after();
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t o[32];
-            const uint32_t ta = tmem + lane_base + kColO + 32 * c2;
-            tmem_ld32(ta, o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(ta, o);
-          }
-        }
-      }
+      // O (rescaled when a row's reference moved) and P's buffer are free
+      // once the previous tile's PV is done: the exponentials and the E4M3
+      // parts below run while it is in flight, and the wait comes after them
       // p = 2^(x - m + 8) -> E4M3 parts, in V's slot order inside each
       // 16-token chunk (word c = slots 2c, 2c+1, 2c+8, 2c+9)
       const float off = 8.f - ((m_run == -INFINITY) ? 0.f : m_run);
@@ -763,11 +757,23 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 #pragma unroll
           for (int q = 0; q < PARTS; ++q) pw[q][cc][c4] = a0[q] | (a1[q] << 16);
         }
-      if (!pv_done) {
+      if (j > 0) {
         ok = tc_wait(pvdone_bar, (uint32_t)((j - 1) & 1), s_abort, limit);
         if (!__all_sync(kFull, ok)) {
           aborted = true;
           break;
+        }
+        if (__any_sync(kFull, move)) {  // rescale the moved rows' O (A7)
+          tc_fence_after();
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_base + kColO + 32 * c2;
+            tmem_ld32(ta, o);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(ta, o);
+          }
         }
       }
 #pragma unroll
