@@ -17,8 +17,9 @@
 // 128.  Six warps:
 //   * warp 4 -- producer: 1-D bulk copies (cp.async.bulk, no multicast) of
 //     the tile's eight 16-token K pieces and eight V pieces (pieces adjacent
-//     in a page go as one copy, one lane per run) into a ring of S stages,
-//     completion on a "full" mbarrier;
+//     in a page go as one copy, one lane per run) into a K ring and a V ring
+//     of S stages each, completion on "full" mbarriers; a K stage is refilled
+//     once the S product has read it, a V stage once the PV product has;
 //   * warp 5, lane 0 -- MMA issuer: per tile
 //       S[64 rows x 128 tok] = (Qhi + Qlo)[64 x 128 d] . K_tile^T
 //     as two M=64, N=64 halves (tokens 0-63 into TMEM lanes 0-15 of each warp
@@ -29,7 +30,8 @@
 //     16-31).  kind::f8f6f4, E4M3 x E4M3, f32 accumulation; the cached codes
 //     are the B operands as they lie in the pages (K rows carry the 128-byte
 //     swizzle, V pages are [d][16 slots] core matrices);
-//   * warps 0-3 -- softmax: thread (warp w, lane l) owns query row
+//   * warps 0-3 -- softmax (those holding at least one of the block's rows;
+//     the others sit out): thread (warp w, lane l) owns query row
 //     16 w + (l % 16) and tokens / head dims 64 (l / 16) .. + 63 of every tile,
 //     reads its S columns with tcgen05.ld, masks, keeps the online-softmax
 //     state (running reference m and sum l, per row), writes P as E4M3 hi + lo
@@ -273,7 +275,7 @@ __host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool t
   t.p = t.q + 2 * (size_t)kOpBytes;                     // P hi, P lo
   t.tab = t.p + (size_t)p_parts(tok_scales) * kOpBytes; // piece table, int32 per 16 tokens
   t.bar = (t.tab + (size_t)max_pieces * 4 + 15) / 16 * 16;
-  t.misc = t.bar + (size_t)(2 * stages + 8) * 8;        // tmem address, abort flag, is_last
+  t.misc = t.bar + (size_t)(5 * stages + 8) * 8;        // tmem address, abort flag, is_last
   t.rows = t.misc + 16;                                 // merge: row reference, denominator
   t.total = t.rows + 2 * kRows * 4 + 1024;              // + slack for 1024-byte alignment
   return t;
@@ -298,14 +300,17 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   uint8_t* sP = smem + lay.p;
   int* s_tab = reinterpret_cast<int*>(smem + lay.tab);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bar);
-  uint64_t* full_bar = bars;              // [S] copies landed
-  uint64_t* empty_bar = bars + S;         // [S] PV of the stage's tile done
-  uint64_t* sfull_bar = bars + 2 * S;     // [2] S buffer written
-  uint64_t* sfree_bar = bars + 2 * S + 2; // [2] S buffer read
-  uint64_t* pfull_bar = bars + 2 * S + 4; // P written (and O rescaled)
-  uint64_t* pvdone_bar = bars + 2 * S + 5;// PV of a tile done
-  uint64_t* drain_bar = bars + 2 * S + 6; // every MMA of the CTA done
-  uint64_t* qready_bar = bars + 2 * S + 7; // Q written
+  uint64_t* kfull_bar = bars;              // [S] K copies landed
+  uint64_t* vfull_bar = bars + S;          // [S] V copies landed
+  uint64_t* kempty_bar = bars + 2 * S;     // [S] S product of the stage's tile done
+  uint64_t* vempty_bar = bars + 3 * S;     // [S] PV product of the stage's tile done
+  uint64_t* sfull_bar = bars + 4 * S;      // [2] S buffer written
+  uint64_t* sfree_bar = bars + 4 * S + 2;  // [2] S buffer read
+  uint64_t* pfull_bar = bars + 4 * S + 4;  // P written (and O rescaled)
+  uint64_t* pvdone_bar = bars + 4 * S + 5; // PV of a tile done
+  uint64_t* drain_bar = bars + 4 * S + 6;  // every MMA of the CTA done
+  uint64_t* qready_bar = bars + 4 * S + 7; // Q written
+  uint64_t* kscfree_bar = bars + 4 * S + 8; // [S] TS: the softmax has read the K scales
   constexpr int PARTS = p_parts(TS);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + lay.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + lay.misc + 4);
@@ -406,6 +411,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     s_tab[k] = pc;
   }
 
+  // softmax warps that hold at least one of the block's rows; the others
+  // (and their rows of Q, S, P and O) sit the tiles out
+  const int n_act = min(4, (rows + 15) / 16);
   const int my_row = 16 * (warp & 3) + (lane & 15);  // softmax warps: this thread's row
   const int my_half = lane >> 4;                     // tokens / dims 64 * half .. + 63
   float row_scale2 = 0.f;                            // score -> base-2 exponent
@@ -413,17 +421,20 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&kfull_bar[s], 1);
+      mbar_init(&vfull_bar[s], 1);
+      mbar_init(&kempty_bar[s], 1);
+      mbar_init(&vempty_bar[s], 1);
+      mbar_init(&kscfree_bar[s], 32 * n_act);
     }
     mbar_init(&sfull_bar[0], 1);
     mbar_init(&sfull_bar[1], 1);
-    mbar_init(&sfree_bar[0], 128);
-    mbar_init(&sfree_bar[1], 128);
-    mbar_init(pfull_bar, 128);
+    mbar_init(&sfree_bar[0], 32 * n_act);
+    mbar_init(&sfree_bar[1], 32 * n_act);
+    mbar_init(pfull_bar, 32 * n_act);
     mbar_init(pvdone_bar, 1);
     mbar_init(drain_bar, 1);
-    mbar_init(qready_bar, 128);
+    mbar_init(qready_bar, 32 * n_act);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -439,87 +450,107 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    // The whole warp: lane 0 waits for the stage and posts the byte count,
-    // then lanes 0-7 (K) and 8-15 (V) each issue the copy of one run of
-    // pieces that lie back to back in the page arrays (a page of 64 slots is
-    // four adjacent pieces), so the tile's copies go out in one instruction.
-    // A token-scale copy (64 bytes per piece) goes with every piece.
-    int issued = 0;
-    const int pc_l = lane & 7;
-    const bool is_v_lane = (lane & 8) != 0;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int st = j % S;
-      bool ok = true;
-      if (j >= S && lane == 0)
-        ok = tc_wait(&empty_bar[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
-      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      issued = j + 1;
-      if (p.test_skip_unit == j && cid == 0) continue;  // lost copy (tests only)
-      // this lane's piece and the run of adjacent pieces it starts
-      const int k = 8 * j + pc_l;
-      const int piece = (k < n_pc) ? s_tab[k] : -1;
-      const int prev = (pc_l > 0 && k - 1 < n_pc) ? s_tab[k - 1] : -2;
-      const bool starts = piece >= 0 && !(pc_l > 0 && prev >= 0 && prev + 1 == piece);
-      int run = 0;
-      if (starts) {
-        run = 1;
-        while (pc_l + run < 8 && k + run < n_pc && s_tab[k + run] == piece + run) ++run;
-      }
-      unsigned valid_mask = __ballot_sync(kFull, piece >= 0 && lane < 8);
-      const uint32_t bytes = (uint32_t)__popc(valid_mask) * (2 * kPiece + (TS ? 2 * 64 : 0));
-      if (lane == 0) {
-        if (bytes == 0)
-          mbar_arrive(&full_bar[st]);
-        else
-          mbar_arrive_expect_tx(&full_bar[st], bytes);
-      }
-      __syncwarp();
-      if (bytes != 0 && lane < 16 && starts) {
-        uint8_t* dst = (is_v_lane ? sV : sK) + (size_t)st * kTileBytes + pc_l * kPiece;
-        const uint8_t* src = (is_v_lane ? p.v_pages : p.k_pages) + (size_t)piece * kPiece;
-        bulk_load(dst, src, (uint32_t)run * kPiece, &full_bar[st]);
-        if constexpr (TS) {  // the run's K or V scales (64 bytes per piece)
-          bulk_load(sTS + (size_t)st * 2 * kTile + (is_v_lane ? kTile : 0) + 16 * pc_l,
-                    (is_v_lane ? p.v_tok_scale : p.k_tok_scale) + (size_t)piece * 16,
-                    (uint32_t)run * 64, &full_bar[st]);
+    // Two groups of eight lanes, K (lanes 0-7) and V (lanes 8-15), each its
+    // own ring: a K stage is refilled as soon as the S product has read it,
+    // a V stage once the PV product has.  In a group, the leader waits for
+    // the stage and posts the byte count, then each lane that starts a run
+    // of pieces lying back to back in the page arrays (a page of 64 slots is
+    // four adjacent pieces) issues one copy for the run, so the group's
+    // copies for a tile go out together.  A token-scale copy (64 bytes per
+    // piece) goes with every piece.
+    if (lane < 16) {
+      const bool kg = lane < 8;
+      const int gl = lane & 7, leader = kg ? 0 : 8;
+      const unsigned gm = kg ? 0x000000FFu : 0x0000FF00u;
+      uint64_t* fullb = kg ? kfull_bar : vfull_bar;
+      uint64_t* emptyb = kg ? kempty_bar : vempty_bar;
+      uint8_t* ring = kg ? sK : sV;
+      const uint8_t* pages = kg ? p.k_pages : p.v_pages;
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % S;
+        bool ok = true;
+        if (j >= S && gl == 0) {
+          ok = tc_wait(&emptyb[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
+          // TS: the K scales of the stage are read by the softmax, after the S product
+          if (TS && kg && ok)
+            ok = tc_wait(&kscfree_bar[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
+        }
+        ok = __shfl_sync(gm, ok ? 1 : 0, leader) != 0;
+        if (!ok) break;
+        issued = j + 1;
+        if (p.test_skip_unit == j && cid == 0) continue;  // lost copy (tests only)
+        // this lane's piece and the run of adjacent pieces it starts
+        const int k = 8 * j + gl;
+        const int piece = (k < n_pc) ? s_tab[k] : -1;
+        const int prev = (gl > 0 && k - 1 < n_pc) ? s_tab[k - 1] : -2;
+        const bool starts = piece >= 0 && !(gl > 0 && prev >= 0 && prev + 1 == piece);
+        int run = 0;
+        if (starts) {
+          run = 1;
+          while (gl + run < 8 && k + run < n_pc && s_tab[k + run] == piece + run) ++run;
+        }
+        const unsigned valid_mask = __ballot_sync(gm, piece >= 0);
+        const uint32_t bytes = (uint32_t)__popc(valid_mask) * (kPiece + (TS ? 64 : 0));
+        if (gl == 0) {
+          if (bytes == 0)
+            mbar_arrive(&fullb[st]);
+          else
+            mbar_arrive_expect_tx(&fullb[st], bytes);
+        }
+        __syncwarp(gm);
+        if (starts) {
+          bulk_load(ring + (size_t)st * kTileBytes + gl * kPiece, pages + (size_t)piece * kPiece,
+                    (uint32_t)run * kPiece, &fullb[st]);
+          if constexpr (TS) {  // the run's K or V scales (64 bytes per piece)
+            bulk_load(sTS + (size_t)st * 2 * kTile + (kg ? 0 : kTile) + 16 * gl,
+                      (kg ? p.k_tok_scale : p.v_tok_scale) + (size_t)piece * 16,
+                      (uint32_t)run * 64, &fullb[st]);
+          }
         }
       }
-    }
-    if (*s_abort && lane == 0) {
-      // drain: copies of the last stages issued may still be in flight
-      for (int j = max(0, issued - S); j < issued; ++j)
-        mbar_wait_bounded(&full_bar[j % S], (uint32_t)((j / S) & 1), limit);
+      if (*s_abort && gl == 0) {
+        // drain: copies of the last stages issued may still be in flight
+        for (int j = max(0, issued - S); j < issued; ++j)
+          mbar_wait_bounded(&fullb[j % S], (uint32_t)((j / S) & 1), limit);
+      }
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f8(64, 64);
-      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // operand descriptors of the first tile, stage 0; every other operand
+      // is one of these plus a byte offset / 16 in the start-address field
+      // (all addresses stay below 256 KB, so the field never carries)
+      const uint64_t dq = smem_desc(smem_u32(sQ), 128, 1024, 0);
+      const uint64_t dp = smem_desc(smem_u32(sP), 128, 1024, 0);
+      const uint64_t dk = smem_desc(smem_u32(sK), 16, 1024, 2);
+      const uint64_t dv = smem_desc(smem_u32(sV), kPiece, 128, 0);
       bool ok = tc_wait(qready_bar, 0, s_abort, limit);
       auto issue_pv = [&](int k) {  // O += P . V for tile k
         const int st = k % S;
         const int tok = t_end - (t_begin + kTile * k);  // valid tokens of the tile (>= 1)
         const int nks = min(4, (tok + 31) / 32);       // 32-token k-steps holding any
+        const uint64_t dvs = dv + (uint64_t)((st * kTileBytes) >> 4);
 #pragma unroll
         for (int dh = 0; dh < 2; ++dh) {
           const uint32_t d = tmem + ((uint32_t)(16 * dh) << 16) + kColO;
 #pragma unroll
           for (int part = 0; part < PARTS; ++part)
-            for (int ks = 0; ks < nks; ++ks) {
-              const uint64_t a =
-                  smem_desc(p_addr + part * kOpBytes + ks * 256, 128, 1024, 0);
-              const uint64_t bd = smem_desc(
-                  v_addr + st * kTileBytes + ks * 2 * kPiece + dh * 1024, kPiece, 128, 0);
-              mma_f8(d, a, bd, idesc, (k > 0 || part > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              if (ks >= nks) break;
+              mma_f8(d, dp + (uint64_t)((part * kOpBytes + ks * 256) >> 4),
+                     dvs + (uint64_t)((ks * 2 * kPiece + dh * 1024) >> 4), idesc,
+                     (k > 0 || part > 0 || ks > 0) ? 1u : 0u);
             }
         }
-        mma_commit(&empty_bar[st]);
+        mma_commit(&vempty_bar[st]);
         mma_commit(pvdone_bar);
       };
       auto issue_s = [&](int j) {  // S = (Qhi + Qlo) . K^T for tile j
         const int st = j % S, sb = j & 1;
+        const uint64_t dks = dk + (uint64_t)((st * kTileBytes) >> 4);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (t_begin + kTile * j + 64 * half >= t_end) break;  // no token in this half
@@ -527,33 +558,34 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
 #pragma unroll
           for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t a = smem_desc(q_addr + part * kOpBytes + ks * 256, 128, 1024, 0);
-              const uint64_t bd =
-                  smem_desc(k_addr + st * kTileBytes + half * 8192 + ks * 32, 16, 1024, 2);
-              mma_f8(d, a, bd, idesc, (part > 0 || ks > 0) ? 1u : 0u);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f8(d, dq + (uint64_t)((part * kOpBytes + ks * 256) >> 4),
+                     dks + (uint64_t)((half * 8192 + ks * 32) >> 4), idesc,
+                     (part > 0 || ks > 0) ? 1u : 0u);
         }
+        mma_commit(&kempty_bar[st]);
         mma_commit(&sfull_bar[sb]);
       };
-      // Event loop: S(js) once tile js has landed and its S buffer is free
-      // (at most two S tiles ahead of the PV products), PV(jp) once the
-      // softmax has written P(jp) -- whichever is ready first, so that a PV
-      // never waits behind the next tile's copies.  Bounded: no progress for
+      // Event loop: S(js) once the K of tile js has landed and its S buffer
+      // is free (at most two S tiles ahead of the PV products), PV(jp) once
+      // the softmax has written P(jp) and the V of tile jp has landed --
+      // whichever is ready first, so that a PV never waits behind the next
+      // tile's copies.  Bounded: no progress for
       // the wait limit raises the abort flag.
       int js = 0, jp = 0;
       uint64_t t_idle = global_timer_ns();
       while (ok && jp < n_tiles) {
         bool progressed = false;
         if (js < n_tiles && js < jp + 2 &&
-            mbar_test(&full_bar[js % S], (uint32_t)((js / S) & 1)) &&
+            mbar_test(&kfull_bar[js % S], (uint32_t)((js / S) & 1)) &&
             (js < 2 || mbar_test(&sfree_bar[js & 1], (uint32_t)(((js >> 1) - 1) & 1)))) {
           tc_fence_after();
           issue_s(js);
           ++js;
           progressed = true;
         }
-        if (jp < js && mbar_test(pfull_bar, (uint32_t)(jp & 1))) {
+        if (jp < js && mbar_test(pfull_bar, (uint32_t)(jp & 1)) &&
+            mbar_test(&vfull_bar[jp % S], (uint32_t)((jp / S) & 1))) {
           tc_fence_after();
           issue_pv(jp);
           ++jp;
@@ -574,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       mma_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, limit);
     }
-  } else {
+  } else if (warp < n_act) {
     // ------------------------------------------------------------ softmax
     // (first the Q rows, while the producer's first copies are in flight)
   // ---- Q rows as E4M3 hi + lo with a per-row power-of-two scale, in the
@@ -664,14 +696,15 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       tc_fence_before();
       mbar_arrive(&sfree_bar[sb]);
 
-      // mask (A5): tokens past the split, in a bad page, or after the row's limit
+      // mask (A5): tokens past the split, in a bad page, or after the row's
+      // limit (a row past the block's rows has limit -1: all masked)
       const int t0 = t_begin + kTile * j + 64 * my_half;
+      const int lim = min(t_end - 1, row_lim);
       float x[64];
-      bool clean = row_ok && (t0 + 63 < t_end) && (t0 + 63 <= row_lim);
-      if (clean) {
+      bool pc_ok[4];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) clean &= s_tab[(t0 - t_begin) / 16 + q4] >= 0;
-      }
+      for (int q4 = 0; q4 < 4; ++q4) pc_ok[q4] = s_tab[(t0 - t_begin) / 16 + q4] >= 0;
+      const bool clean = (t0 + 63 <= lim) && pc_ok[0] && pc_ok[1] && pc_ok[2] && pc_ok[3];
       if constexpr (TS) {  // per-token K scales
         const float4* ksc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile +
                                                              64 * my_half);
@@ -683,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           sv[4 * k4 + 2] = __float_as_uint(__uint_as_float(sv[4 * k4 + 2]) * f.z);
           sv[4 * k4 + 3] = __float_as_uint(__uint_as_float(sv[4 * k4 + 3]) * f.w);
         }
+        mbar_arrive(&kscfree_bar[st]);  // the K producer may refill the stage
       }
       if (clean) {
 #pragma unroll
@@ -690,9 +724,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       } else {
 #pragma unroll
         for (int k = 0; k < 64; ++k) {
-          const int t = t0 + k;
-          const bool ok_t = row_ok && t < t_end && t <= row_lim &&
-                            s_tab[(t - t_begin) >> 4] >= 0;
+          const bool ok_t = t0 + k <= lim && pc_ok[k >> 4];
           x[k] = ok_t ? __uint_as_float(sv[k]) * row_scale2 : -INFINITY;
         }
       }
@@ -732,6 +764,11 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       }
       l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       if constexpr (TS) {  // p * v_scale[t] / bound: at most p (masked tokens stay 0)
+        ok = tc_wait(&vfull_bar[st], (uint32_t)((j / S) & 1), s_abort, limit);  // V scales
+        if (!__all_sync(kFull, ok)) {
+          aborted = true;
+          break;
+        }
         const float inv_bound = 1.f / v_scale;
         const float4* vsc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile + kTile +
                                                              64 * my_half);
@@ -794,21 +831,23 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         dirty |= (k < n_pc && s_tab[k] < 0);
       }
       if (dirty) {
-        ok = tc_wait(&full_bar[st], (uint32_t)((j / S) & 1), s_abort, limit);
+        ok = tc_wait(&vfull_bar[st], (uint32_t)((j / S) & 1), s_abort, limit);
         if (!__all_sync(kFull, ok)) {
           aborted = true;
           break;
         }
-        const int d = tid;  // 0..127: one V row of every piece
-        for (int pc = 0; pc < 8; ++pc) {
-          const int k = 8 * j + pc;
-          const int nvalid = (k < n_pc && s_tab[k] >= 0) ? min(16, t_end - (tile0 + 16 * pc)) : 0;
-          if (nvalid >= 16) continue;
-          uint8_t* vrow = sV + (size_t)st * kTileBytes + pc * kPiece + d * 16;
-          if (nvalid <= 0) {
-            *reinterpret_cast<uint4*>(vrow) = make_uint4(0u, 0u, 0u, 0u);
-          } else {
-            for (int t = nvalid; t < 16; ++t) vrow[group_pos(t)] = 0;
+        for (int d = tid; d < kD; d += 32 * n_act) {  // one V row of every piece
+          for (int pc = 0; pc < 8; ++pc) {
+            const int k = 8 * j + pc;
+            const int nvalid =
+                (k < n_pc && s_tab[k] >= 0) ? min(16, t_end - (tile0 + 16 * pc)) : 0;
+            if (nvalid >= 16) continue;
+            uint8_t* vrow = sV + (size_t)st * kTileBytes + pc * kPiece + d * 16;
+            if (nvalid <= 0) {
+              *reinterpret_cast<uint4*>(vrow) = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+              for (int t = nvalid; t < 16; ++t) vrow[group_pos(t)] = 0;
+            }
           }
         }
       }
