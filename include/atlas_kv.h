@@ -161,6 +161,8 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
 /* Tuning options for atlas_kv_pool_set_option. */
 #define ATLAS_OPT_SPLIT_TOKENS   1   /* same as atlas_kv_pool_set_split_tokens           */
 #define ATLAS_OPT_STAGES         2   /* K/V staging depth per stream: 0 = auto, 2 or 3   */
+                                     /* (tensor-core kernel: depth of the K ring, auto 3; */
+                                     /* its V ring always has 2 stages)                  */
 #define ATLAS_OPT_WAVES          3   /* automatic sizing, 0 = 1, up to 8: balanced: CTAs */
                                      /* per resident CTA slot; grid: splits sized for     */
                                      /* 2 x this many waves of resident CTAs; more, smaller */
@@ -183,9 +185,11 @@ ATLAS_API atlas_status_t atlas_kv_pool_set_split_tokens(atlas_kv_pool_t* pool, i
                                      /* runs blocks of 64 query rows in the grid         */
                                      /* partition (ATLAS_OPT_PARTITION and              */
                                      /* ATLAS_OPT_ROWS_PER_CTA do not apply to it)      */
-#define ATLAS_OPT_WAIT_LIMIT_US  6   /* wall-clock limit of every bounded wait inside the */
-                                     /* decode kernel, in microseconds: 0 = the default  */
-                                     /* (200 ms), else 1 .. 10^7                          */
+#define ATLAS_OPT_WAIT_LIMIT_US  6   /* limit of every bounded wait inside the decode  */
+                                     /* kernel, in microseconds: 0 = the default        */
+                                     /* (200 ms), else 1 .. 10^7.  Counted in SM cycles */
+                                     /* at 2 per ns: at least this long at any SM clock */
+                                     /* up to 2 GHz, longer at a lower clock            */
 #define ATLAS_OPT_TEST_SKIP_UNIT 7   /* TESTS ONLY: -1 = off (default); k >= 0 = the     */
                                      /* first K/V stream of CTA 0 never issues the copies */
                                      /* of its k-th unit (tensor-core kernel: of its k-th */

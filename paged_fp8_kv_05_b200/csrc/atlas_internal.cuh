@@ -160,7 +160,7 @@ inline DecodeLaunch plan_decode_tc(int B, int Hq, int Hkv, int q_len, int max_se
   L.rbg = 4;
   L.rows_per_cta = 64;
   L.row_blocks = (R + 63) / 64;
-  L.stages = stages_override > 0 ? stages_override : 2;
+  L.stages = stages_override > 0 ? stages_override : 3;  // K ring depth (the V ring has 2)
   L.segs = (long long)B * Hkv * L.row_blocks;
   L.units_max = L.segs * (((long long)max_seq_len + 31) / 32);
   L.grid_mode = 1;
@@ -296,7 +296,7 @@ cudaError_t launch_decode_fp8(const DecodeParams& p, int rows_per_warp, int rbg,
                               long long grid, cudaStream_t stream);
 
 // Tensor-core decode kernel (head_dim 128): 1-D grid of `grid` CTAs, one per
-// (segment, split); stages 2 or 3.
+// (segment, split); stages = the K ring's depth, 2 or 3 (the V ring has 2).
 cudaError_t launch_decode_tc(const DecodeParams& p, int stages, long long grid,
                              cudaStream_t stream);
 size_t decode_tc_smem_bytes(int stages, int split_tokens, bool tok_scales);
@@ -458,13 +458,23 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Wait for an mbarrier phase with a wall-clock limit; false if it ran out.
+// This SM's cycle counter.  Bounded waits measure with it rather than with
+// the global nanosecond timer, which is far slower to read: a wait loop that
+// reads that timer on every pass delays the hand-offs it waits for.
+__device__ __forceinline__ uint64_t sm_cycles() { return (uint64_t)clock64(); }
+
+// A wait limit in nanoseconds as SM cycles, at two cycles per nanosecond: at
+// least the limit at any SM clock up to 2 GHz (a slower clock only stretches
+// it).
+__device__ __forceinline__ uint64_t ns_to_cycles(uint64_t ns) { return 2 * ns; }
+
+// Wait for an mbarrier phase with a time limit; false if it ran out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = sm_cycles(), limit = ns_to_cycles(limit_ns);
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > limit_ns) return false;
+    if (sm_cycles() - t0 > limit) return false;
   }
   return true;
 }
@@ -472,15 +482,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 // 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses
 // 16-byte aligned), completion counted on `bar` (no multicast).  The KV pages
 // are read once per call: the L2 lines they fill are marked evict-first.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t policy;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1], %2, [%3], %4;"
       ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  bulk_load(dst, src, bytes, bar, l2_evict_first_policy());
 }
 
 #endif  // __CUDACC__

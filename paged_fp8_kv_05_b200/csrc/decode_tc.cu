@@ -64,9 +64,11 @@ constexpr int kD = 128;                    // head dim
 constexpr int kPiece = 16 * kD;            // one 16-token K or V piece: 2048 bytes
 constexpr int kTileBytes = 8 * kPiece;     // K (or V) of one tile: 16 KB
 constexpr int kOpBytes = kRows * kD;       // one E4M3 part of Q or P: 8 KB
+constexpr int kVS = 2;                     // V ring stages (the K ring has KS)
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;              // S double buffer: columns 0-63, 64-127
 constexpr uint32_t kColO = 128;            // O: columns 128-191
+constexpr uint32_t kColQ = 192;            // Q hi: 192-223, Q lo: 224-255 (A operand)
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---------------------------------------------------------------- tcgen05 PTX
@@ -100,6 +102,20 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]^T, kind::f8f6f4, A read from tensor memory.
+// With M = 64, row m of A sits in the same lane as row m of D (lanes 0-15 of
+// each 32-lane quadrant, or 16-31 at lane offset 16), its K = 32 E4M3 values
+// in 8 consecutive 32-bit columns, 4 per column in byte order.
+__device__ __forceinline__ void mma_f8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -243,13 +259,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Bounded wait that also gives up when another role has flagged an abort;
 // a wait that runs out raises the abort flag.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                        uint64_t limit_ns) {
+                                        uint64_t limit_cycles) {
   if (mbar_probe(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = sm_cycles();
   while (true) {
     if (mbar_probe(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
+    if (sm_cycles() - t0 > limit_cycles) {
       *abort_flag = 1;
       return false;
     }
@@ -259,25 +275,29 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // ----------------------------------------------------------- shared memory
 
 struct TcLayout {
-  size_t k, v, ts, q, p, tab, bar, misc, rows, total;
+  size_t k, v, ts, p, tab, bar, misc, rows, total;
 };
 // E4M3 parts that carry a probability into the PV product: hi + lo (8
 // significant bits); three with per-token V scales, where even the row's
 // largest probability is no longer a power of two
 __host__ __device__ constexpr int p_parts(bool tok_scales) { return tok_scales ? 3 : 2; }
-// ts: per-token K and V scales of each stage (finer-grained mode), else empty
-__host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool tok_scales) {
+// barriers: K ring full / empty / scales-read (KS each), V ring full / empty
+// (kVS each), S buffers full / free (2 each), P full, PV done, drain, Q ready
+__host__ __device__ constexpr int tc_barriers(int k_stages) { return 3 * k_stages + 2 * kVS + 8; }
+// ts: per-token K scales of each K stage and V scales of each V stage
+// (finer-grained mode), else empty
+__host__ __device__ inline TcLayout tc_layout(int k_stages, int max_pieces, bool tok_scales) {
   TcLayout t;
-  t.k = 0;                                              // [S][8 pieces][16 tok][128 B] (swizzled)
-  t.v = t.k + (size_t)stages * kTileBytes;              // [S][8 pieces][128 d][16 slots]
-  t.ts = t.v + (size_t)stages * kTileBytes;             // [S][K, V][128 tokens] float32
-  t.q = t.ts + (tok_scales ? (size_t)stages * 2 * kTile * 4 : 0);  // Q hi, Q lo: core matrices
-  t.p = t.q + 2 * (size_t)kOpBytes;                     // P hi, P lo
+  t.k = 0;                                              // [KS][8 pieces][16 tok][128 B] (swizzled)
+  t.v = t.k + (size_t)k_stages * kTileBytes;            // [kVS][8 pieces][128 d][16 slots]
+  t.ts = t.v + (size_t)kVS * kTileBytes;                // [KS][128] K scales, [kVS][128] V scales
+  t.p = t.ts + (tok_scales ? (size_t)(k_stages + kVS) * kTile * 4 : 0);  // P parts: core matrices
   t.tab = t.p + (size_t)p_parts(tok_scales) * kOpBytes; // piece table, int32 per 16 tokens
   t.bar = (t.tab + (size_t)max_pieces * 4 + 15) / 16 * 16;
-  t.misc = t.bar + (size_t)(5 * stages + 8) * 8;        // tmem address, abort flag, is_last
-  t.rows = t.misc + 16;                                 // merge: row reference, denominator
-  t.total = t.rows + 2 * kRows * 4 + 1024;              // + slack for 1024-byte alignment
+  t.misc = t.bar + (size_t)tc_barriers(k_stages) * 8;   // tmem address, abort flag, is_last
+  t.rows = t.k;                                         // merge: row reference, denominator
+                                                        // (after the tiles: K stage 0)
+  t.total = t.misc + 16 + 1024;                         // + slack for 1024-byte alignment
   return t;
 }
 
@@ -288,29 +308,29 @@ __host__ __device__ inline TcLayout tc_layout(int stages, int max_pieces, bool t
 // codes; K scales multiply the scores, V scales (divided by the head's bound
 // p.v_scale[h], so that the probabilities stay in E4M3 range) the
 // probabilities of the PV product, and the bound scales the output.
-template <int S, bool TS>
+template <int KS, bool TS>
 __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const TcLayout lay = tc_layout(S, p.split_tokens / 16, TS);
-  float* sTS = reinterpret_cast<float*>(smem + lay.ts);  // [S][2][128]
+  const TcLayout lay = tc_layout(KS, p.split_tokens / 16, TS);
+  float* sKS = reinterpret_cast<float*>(smem + lay.ts);  // [KS][128] K scales
+  float* sVS = sKS + KS * kTile;                          // [kVS][128] V scales
   uint8_t* sK = smem + lay.k;
   uint8_t* sV = smem + lay.v;
-  uint8_t* sQ = smem + lay.q;
   uint8_t* sP = smem + lay.p;
   int* s_tab = reinterpret_cast<int*>(smem + lay.tab);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bar);
-  uint64_t* kfull_bar = bars;              // [S] K copies landed
-  uint64_t* vfull_bar = bars + S;          // [S] V copies landed
-  uint64_t* kempty_bar = bars + 2 * S;     // [S] S product of the stage's tile done
-  uint64_t* vempty_bar = bars + 3 * S;     // [S] PV product of the stage's tile done
-  uint64_t* sfull_bar = bars + 4 * S;      // [2] S buffer written
-  uint64_t* sfree_bar = bars + 4 * S + 2;  // [2] S buffer read
-  uint64_t* pfull_bar = bars + 4 * S + 4;  // P written (and O rescaled)
-  uint64_t* pvdone_bar = bars + 4 * S + 5; // PV of a tile done
-  uint64_t* drain_bar = bars + 4 * S + 6;  // every MMA of the CTA done
-  uint64_t* qready_bar = bars + 4 * S + 7; // Q written
-  uint64_t* kscfree_bar = bars + 4 * S + 8; // [S] TS: the softmax has read the K scales
+  uint64_t* kfull_bar = bars;                  // [KS] K copies landed
+  uint64_t* kempty_bar = kfull_bar + KS;       // [KS] S product of the stage's tile done
+  uint64_t* kscfree_bar = kempty_bar + KS;     // [KS] TS: the softmax has read the K scales
+  uint64_t* vfull_bar = kscfree_bar + KS;      // [kVS] V copies landed
+  uint64_t* vempty_bar = vfull_bar + kVS;      // [kVS] PV product of the stage's tile done
+  uint64_t* sfull_bar = vempty_bar + kVS;      // [2] S buffer written
+  uint64_t* sfree_bar = sfull_bar + 2;         // [2] S buffer read
+  uint64_t* pfull_bar = sfree_bar + 2;         // P written (and O rescaled)
+  uint64_t* pvdone_bar = pfull_bar + 1;        // PV of a tile done
+  uint64_t* drain_bar = pvdone_bar + 1;        // every MMA of the CTA done
+  uint64_t* qready_bar = drain_bar + 1;        // Q written to tensor memory
   constexpr int PARTS = p_parts(TS);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + lay.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + lay.misc + 4);
@@ -420,12 +440,14 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   int row_lim = -1;                                  // last visible key position
   if (tid == 0) {
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&kfull_bar[s], 1);
-      mbar_init(&vfull_bar[s], 1);
       mbar_init(&kempty_bar[s], 1);
-      mbar_init(&vempty_bar[s], 1);
       mbar_init(&kscfree_bar[s], 32 * n_act);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(&vfull_bar[s], 1);
+      mbar_init(&vempty_bar[s], 1);
     }
     mbar_init(&sfull_bar[0], 1);
     mbar_init(&sfull_bar[1], 1);
@@ -446,74 +468,98 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
   __syncthreads();  // table, barriers, tensor memory and appended tokens ready
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint64_t limit = p.wait_limit_ns;
+  const uint64_t limit = ns_to_cycles(p.wait_limit_ns);  // for tc_wait and the event loops
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    // Two groups of eight lanes, K (lanes 0-7) and V (lanes 8-15), each its
-    // own ring: a K stage is refilled as soon as the S product has read it,
-    // a V stage once the PV product has.  In a group, the leader waits for
-    // the stage and posts the byte count, then each lane that starts a run
-    // of pieces lying back to back in the page arrays (a page of 64 slots is
-    // four adjacent pieces) issues one copy for the run, so the group's
-    // copies for a tile go out together.  A token-scale copy (64 bytes per
-    // piece) goes with every piece.
-    if (lane < 16) {
-      const bool kg = lane < 8;
-      const int gl = lane & 7, leader = kg ? 0 : 8;
-      const unsigned gm = kg ? 0x000000FFu : 0x0000FF00u;
-      uint64_t* fullb = kg ? kfull_bar : vfull_bar;
-      uint64_t* emptyb = kg ? kempty_bar : vempty_bar;
-      uint8_t* ring = kg ? sK : sV;
-      const uint8_t* pages = kg ? p.k_pages : p.v_pages;
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % S;
-        bool ok = true;
-        if (j >= S && gl == 0) {
-          ok = tc_wait(&emptyb[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
-          // TS: the K scales of the stage are read by the softmax, after the S product
-          if (TS && kg && ok)
-            ok = tc_wait(&kscfree_bar[st], (uint32_t)(((j / S) - 1) & 1), s_abort, limit);
-        }
-        ok = __shfl_sync(gm, ok ? 1 : 0, leader) != 0;
-        if (!ok) break;
-        issued = j + 1;
-        if (p.test_skip_unit == j && cid == 0) continue;  // lost copy (tests only)
-        // this lane's piece and the run of adjacent pieces it starts
-        const int k = 8 * j + gl;
-        const int piece = (k < n_pc) ? s_tab[k] : -1;
-        const int prev = (gl > 0 && k - 1 < n_pc) ? s_tab[k - 1] : -2;
-        const bool starts = piece >= 0 && !(gl > 0 && prev >= 0 && prev + 1 == piece);
-        int run = 0;
-        if (starts) {
-          run = 1;
-          while (gl + run < 8 && k + run < n_pc && s_tab[k + run] == piece + run) ++run;
-        }
-        const unsigned valid_mask = __ballot_sync(gm, piece >= 0);
-        const uint32_t bytes = (uint32_t)__popc(valid_mask) * (kPiece + (TS ? 64 : 0));
-        if (gl == 0) {
-          if (bytes == 0)
-            mbar_arrive(&fullb[st]);
-          else
-            mbar_arrive_expect_tx(&fullb[st], bytes);
-        }
-        __syncwarp(gm);
-        if (starts) {
-          bulk_load(ring + (size_t)st * kTileBytes + gl * kPiece, pages + (size_t)piece * kPiece,
-                    (uint32_t)run * kPiece, &fullb[st]);
-          if constexpr (TS) {  // the run's K or V scales (64 bytes per piece)
-            bulk_load(sTS + (size_t)st * 2 * kTile + (kg ? 0 : kTile) + 16 * gl,
-                      (kg ? p.k_tok_scale : p.v_tok_scale) + (size_t)piece * 16,
-                      (uint32_t)run * 64, &fullb[st]);
+    // One converged warp serves two rings, K and V: a K stage is refilled as
+    // soon as the S product has read it (and, with per-token scales, the
+    // softmax has read its K scales), a V stage once the PV product has.
+    // Each pass, lanes 0-2 test the three release barriers at once; then
+    // lanes 0-7 take the K pieces of tile jk and lanes 8-15 the V pieces of
+    // tile jv (either group only if its stage is free), and every lane that
+    // starts a run of pieces lying back to back in the page arrays (a page of
+    // 64 slots is four adjacent pieces) issues one copy for the run: a
+    // tile's copies go out together, with no serial work per piece.  A
+    // token-scale copy (64 bytes per piece) goes with every piece.  Bounded:
+    // no progress for the wait limit raises the abort flag.
+    const uint64_t policy = l2_evict_first_policy();
+    const bool kg = lane < 8;
+    const int gl = lane & 7;
+    int jk = 0, jv = 0;
+    uint64_t t_idle = sm_cycles();
+    while (jk < n_tiles || jv < n_tiles) {
+      bool rdy = false;
+      if (lane == 0)
+        rdy = jk < n_tiles &&
+              (jk < KS || mbar_test(&kempty_bar[jk % KS], (uint32_t)(((jk / KS) - 1) & 1)));
+      else if (lane == 1)
+        rdy = !TS || jk >= n_tiles || jk < KS ||
+              mbar_test(&kscfree_bar[jk % KS], (uint32_t)(((jk / KS) - 1) & 1));
+      else if (lane == 2)
+        rdy = jv < n_tiles &&
+              (jv < kVS || mbar_test(&vempty_bar[jv % kVS], (uint32_t)(((jv / kVS) - 1) & 1)));
+      const unsigned r = __ballot_sync(kFull, rdy);
+      const bool do_k = (r & 3u) == 3u, do_v = (r & 4u) != 0;
+      if (!do_k && !do_v) {
+        bool stop = false;
+        if (lane == 0) {
+          if (*s_abort) {
+            stop = true;
+          } else if (sm_cycles() - t_idle > limit) {
+            *s_abort = 1;
+            stop = true;
           }
         }
+        if (__shfl_sync(kFull, stop ? 1 : 0, 0)) break;
+        __nanosleep(32);
+        continue;
       }
-      if (*s_abort && gl == 0) {
-        // drain: copies of the last stages issued may still be in flight
-        for (int j = max(0, issued - S); j < issued; ++j)
-          mbar_wait_bounded(&fullb[j % S], (uint32_t)((j / S) & 1), limit);
+      if (lane == 0) t_idle = sm_cycles();
+      const int j = kg ? jk : jv;
+      const bool mine = lane < 16 && (kg ? do_k : do_v) &&
+                        !(p.test_skip_unit == j && cid == 0);  // lost copy (tests only)
+      const int st = kg ? j % KS : j % kVS;
+      uint64_t* fb = kg ? &kfull_bar[st] : &vfull_bar[st];
+      const int k = 8 * j + gl;
+      const int piece = (mine && k < n_pc) ? s_tab[k] : -1;
+      // a run starts at a valid piece whose left neighbour (same group) is
+      // not the piece before it in the page arrays
+      const int left = __shfl_up_sync(kFull, piece, 1);
+      const bool adj = gl > 0 && piece >= 0 && left >= 0 && left + 1 == piece;
+      const unsigned adj_mask = __ballot_sync(kFull, adj);
+      const unsigned valid_mask = __ballot_sync(kFull, piece >= 0);
+      const bool starts = piece >= 0 && !adj;
+      // run length: this piece plus the adjacent pieces right after it
+      const int run = starts ? __ffs(~(adj_mask >> (lane + 1))) : 0;
+      const unsigned grp_valid = valid_mask & (kg ? 0x000000FFu : 0x0000FF00u);
+      if (mine && gl == 0) {
+        const uint32_t bytes = (uint32_t)__popc(grp_valid) * (kPiece + (TS ? 64 : 0));
+        if (bytes == 0)
+          mbar_arrive(fb);
+        else
+          mbar_arrive_expect_tx(fb, bytes);
       }
+      __syncwarp();
+      if (starts) {
+        bulk_load((kg ? sK : sV) + (size_t)st * kTileBytes + gl * kPiece,
+                  (kg ? p.k_pages : p.v_pages) + (size_t)piece * kPiece, (uint32_t)run * kPiece,
+                  fb, policy);
+        if constexpr (TS) {  // the run's K or V scales (64 bytes per piece)
+          bulk_load((kg ? sKS : sVS) + (size_t)st * kTile + 16 * gl,
+                    (kg ? p.k_tok_scale : p.v_tok_scale) + (size_t)piece * 16,
+                    (uint32_t)run * 64, fb, policy);
+        }
+      }
+      if (do_k) ++jk;
+      if (do_v) ++jv;
+    }
+    if (*s_abort && lane == 0) {
+      // drain: copies of the last stages issued may still be in flight
+      for (int j = max(0, jk - KS); j < jk; ++j)
+        mbar_wait_bounded(&kfull_bar[j % KS], (uint32_t)((j / KS) & 1), p.wait_limit_ns);
+      for (int j = max(0, jv - kVS); j < jv; ++j)
+        mbar_wait_bounded(&vfull_bar[j % kVS], (uint32_t)((j / kVS) & 1), p.wait_limit_ns);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
@@ -522,13 +568,12 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       // operand descriptors of the first tile, stage 0; every other operand
       // is one of these plus a byte offset / 16 in the start-address field
       // (all addresses stay below 256 KB, so the field never carries)
-      const uint64_t dq = smem_desc(smem_u32(sQ), 128, 1024, 0);
       const uint64_t dp = smem_desc(smem_u32(sP), 128, 1024, 0);
       const uint64_t dk = smem_desc(smem_u32(sK), 16, 1024, 2);
       const uint64_t dv = smem_desc(smem_u32(sV), kPiece, 128, 0);
       bool ok = tc_wait(qready_bar, 0, s_abort, limit);
       auto issue_pv = [&](int k) {  // O += P . V for tile k
-        const int st = k % S;
+        const int st = k % kVS;
         const int tok = t_end - (t_begin + kTile * k);  // valid tokens of the tile (>= 1)
         const int nks = min(4, (tok + 31) / 32);       // 32-token k-steps holding any
         const uint64_t dvs = dv + (uint64_t)((st * kTileBytes) >> 4);
@@ -549,19 +594,20 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         mma_commit(pvdone_bar);
       };
       auto issue_s = [&](int j) {  // S = (Qhi + Qlo) . K^T for tile j
-        const int st = j % S, sb = j & 1;
+        const int st = j % KS, sb = j & 1;
         const uint64_t dks = dk + (uint64_t)((st * kTileBytes) >> 4);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (t_begin + kTile * j + 64 * half >= t_end) break;  // no token in this half
-          const uint32_t d = tmem + ((uint32_t)(16 * half) << 16) + kColS + 64 * sb;
+          // Q rows sit in the same lanes as the S rows they produce
+          const uint32_t lanes = (uint32_t)(16 * half) << 16;
 #pragma unroll
           for (int part = 0; part < 2; ++part)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-              mma_f8(d, dq + (uint64_t)((part * kOpBytes + ks * 256) >> 4),
-                     dks + (uint64_t)((half * 8192 + ks * 32) >> 4), idesc,
-                     (part > 0 || ks > 0) ? 1u : 0u);
+              mma_f8_ta(tmem + lanes + kColS + 64 * sb, tmem + lanes + kColQ + 32 * part + 8 * ks,
+                        dks + (uint64_t)((half * 8192 + ks * 32) >> 4), idesc,
+                        (part > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&kempty_bar[st]);
         mma_commit(&sfull_bar[sb]);
@@ -570,14 +616,14 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       // is free (at most two S tiles ahead of the PV products), PV(jp) once
       // the softmax has written P(jp) and the V of tile jp has landed --
       // whichever is ready first, so that a PV never waits behind the next
-      // tile's copies.  Bounded: no progress for
-      // the wait limit raises the abort flag.
+      // tile's copies.  Bounded: no progress for the wait limit raises the
+      // abort flag.
       int js = 0, jp = 0;
-      uint64_t t_idle = global_timer_ns();
+      uint64_t t_idle = sm_cycles();
       while (ok && jp < n_tiles) {
         bool progressed = false;
         if (js < n_tiles && js < jp + 2 &&
-            mbar_test(&kfull_bar[js % S], (uint32_t)((js / S) & 1)) &&
+            mbar_test(&kfull_bar[js % KS], (uint32_t)((js / KS) & 1)) &&
             (js < 2 || mbar_test(&sfree_bar[js & 1], (uint32_t)(((js >> 1) - 1) & 1)))) {
           tc_fence_after();
           issue_s(js);
@@ -585,17 +631,17 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           progressed = true;
         }
         if (jp < js && mbar_test(pfull_bar, (uint32_t)(jp & 1)) &&
-            mbar_test(&vfull_bar[jp % S], (uint32_t)((jp / S) & 1))) {
+            mbar_test(&vfull_bar[jp % kVS], (uint32_t)((jp / kVS) & 1))) {
           tc_fence_after();
           issue_pv(jp);
           ++jp;
           progressed = true;
         }
         if (progressed) {
-          t_idle = global_timer_ns();
+          t_idle = sm_cycles();
         } else if (*s_abort) {
           ok = false;
-        } else if (global_timer_ns() - t_idle > limit) {
+        } else if (sm_cycles() - t_idle > limit) {
           *s_abort = 1;
           ok = false;
         } else {
@@ -604,14 +650,16 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       }
       // every MMA issued so far has completed before tensor memory is released
       mma_commit(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, limit);
+      mbar_wait_bounded(drain_bar, 0, p.wait_limit_ns);
     }
   } else if (warp < n_act) {
     // ------------------------------------------------------------ softmax
     // (first the Q rows, while the producer's first copies are in flight)
-  // ---- Q rows as E4M3 hi + lo with a per-row power-of-two scale, in the
-  // K-major core-matrix layout of the A operand: row r, 16-dim chunk c at
-  // (r / 8) * 1024 + c * 128 + (r % 8) * 16
+  // ---- Q rows as E4M3 hi + lo with a per-row power-of-two scale, written
+  // to tensor memory as the A operand of the S product: row r in the lanes
+  // of the S rows it produces -- both lane r % 16 and lane 16 + r % 16 of
+  // warp r / 16's quadrant, for the two token halves -- dims 4c .. 4c + 3 of
+  // a part in column c (hi: kColQ + c, lo: kColQ + 32 + c)
   {
     const int r = my_row, rr = row0 + r;
     float x[64];
@@ -646,9 +694,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       if (amax * a > 448.f) a *= 0.5f;
     }
     row_scale2 = k_scale * p.qk_scale_log2 / a;
+    uint32_t hw[16], lw[16];  // this thread's 64 dims: word 4 cc + w4 = dims 16 cc + 4 w4 ..
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
-      uint32_t hw[4], lw[4];
 #pragma unroll
       for (int w4 = 0; w4 < 4; ++w4) {
         const int k0 = 16 * cc + 4 * w4;
@@ -659,14 +707,26 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
         const uint32_t l01 = f32x2_to_e4m3x2(y0 - b01.x, y1 - b01.y);
         const uint32_t l23 = f32x2_to_e4m3x2(y2 - b23.x, y3 - b23.y);
-        hw[w4] = h01 | (h23 << 16);
-        lw[w4] = l01 | (l23 << 16);
+        hw[4 * cc + w4] = h01 | (h23 << 16);
+        lw[4 * cc + w4] = l01 | (l23 << 16);
       }
-      const int off = (r >> 3) * 1024 + (4 * my_half + cc) * 128 + (r & 7) * 16;
-      *reinterpret_cast<uint4*>(sQ + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(sQ + kOpBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    fence_proxy_async_shared();  // Q is read by the tensor core
+    // the whole row in this thread's lane: the partner (lane ^ 16) holds the
+    // other 64 dims
+    const uint32_t qa = tmem + ((uint32_t)(32 * warp) << 16) + kColQ;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      uint32_t row[32];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t own = part ? lw[c] : hw[c];
+        const uint32_t other = __shfl_xor_sync(kFull, own, 16);
+        row[c] = my_half ? other : own;
+        row[16 + c] = my_half ? own : other;
+      }
+      tmem_st32(qa + 32 * part, row);
+    }
+    tc_fence_before();
     mbar_arrive(qready_bar);
   }
 
@@ -675,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     float m_run = -INFINITY, l_run = 0.f;
     bool aborted = false;
     for (int j = 0; j < n_tiles; ++j) {
-      const int sb = j & 1, st = j % S;
+      const int sb = j & 1, sk = j % KS, sv_st = j % kVS;
+      const uint32_t vpar = (uint32_t)((j / kVS) & 1);
       bool ok = tc_wait(&sfull_bar[sb], (uint32_t)((j >> 1) & 1), s_abort, limit);
       if (!__all_sync(kFull, ok)) {
         aborted = true;
@@ -706,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       for (int q4 = 0; q4 < 4; ++q4) pc_ok[q4] = s_tab[(t0 - t_begin) / 16 + q4] >= 0;
       const bool clean = (t0 + 63 <= lim) && pc_ok[0] && pc_ok[1] && pc_ok[2] && pc_ok[3];
       if constexpr (TS) {  // per-token K scales
-        const float4* ksc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile +
+        const float4* ksc = reinterpret_cast<const float4*>(sKS + (size_t)sk * kTile +
                                                              64 * my_half);
 #pragma unroll
         for (int k4 = 0; k4 < 16; ++k4) {
@@ -716,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
           sv[4 * k4 + 2] = __float_as_uint(__uint_as_float(sv[4 * k4 + 2]) * f.z);
           sv[4 * k4 + 3] = __float_as_uint(__uint_as_float(sv[4 * k4 + 3]) * f.w);
         }
-        mbar_arrive(&kscfree_bar[st]);  // the K producer may refill the stage
+        mbar_arrive(&kscfree_bar[sk]);  // the K producer may refill the stage
       }
       if (clean) {
 #pragma unroll
@@ -764,13 +825,13 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
       }
       l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       if constexpr (TS) {  // p * v_scale[t] / bound: at most p (masked tokens stay 0)
-        ok = tc_wait(&vfull_bar[st], (uint32_t)((j / S) & 1), s_abort, limit);  // V scales
+        ok = tc_wait(&vfull_bar[sv_st], vpar, s_abort, limit);  // V scales
         if (!__all_sync(kFull, ok)) {
           aborted = true;
           break;
         }
         const float inv_bound = 1.f / v_scale;
-        const float4* vsc = reinterpret_cast<const float4*>(sTS + (size_t)st * 2 * kTile + kTile +
+        const float4* vsc = reinterpret_cast<const float4*>(sVS + (size_t)sv_st * kTile +
                                                              64 * my_half);
 #pragma unroll
         for (int k4 = 0; k4 < 16; ++k4) {
@@ -831,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
         dirty |= (k < n_pc && s_tab[k] < 0);
       }
       if (dirty) {
-        ok = tc_wait(&vfull_bar[st], (uint32_t)((j / S) & 1), s_abort, limit);
+        ok = tc_wait(&vfull_bar[sv_st], vpar, s_abort, limit);
         if (!__all_sync(kFull, ok)) {
           aborted = true;
           break;
@@ -842,7 +903,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
             const int nvalid =
                 (k < n_pc && s_tab[k] >= 0) ? min(16, t_end - (tile0 + 16 * pc)) : 0;
             if (nvalid >= 16) continue;
-            uint8_t* vrow = sV + (size_t)st * kTileBytes + pc * kPiece + d * 16;
+            uint8_t* vrow = sV + (size_t)sv_st * kTileBytes + pc * kPiece + d * 16;
             if (nvalid <= 0) {
               *reinterpret_cast<uint4*>(vrow) = make_uint4(0u, 0u, 0u, 0u);
             } else {
