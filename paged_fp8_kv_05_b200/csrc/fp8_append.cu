@@ -52,9 +52,7 @@ __device__ __forceinline__ float token_row_scale(const float (&x)[16]) {
 template <int D, bool TS>
 __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
   constexpr int CH = D / 16;  // 16-element chunks per row
-  constexpr int NW = D / 32;  // warps
   __shared__ int s_page[kTok];
-  __shared__ float s_amax[NW][kTok];
   const int n_tiles = (p.n_new + kTok - 1) / kTok;
   const int tile = blockIdx.x % n_tiles;
   const int bh = blockIdx.x / n_tiles;
@@ -79,90 +77,105 @@ __global__ void __launch_bounds__(D) fp8_append_kernel(const AppendParams p) {
     s_page[tid] = page;
   }
 
-  // ---- V, one head dimension per thread: element d of the tile's 16 tokens
-  // (each load instruction reads one token's row across the CTA: coalesced),
-  // quantised and packed in the 16-slot group order -- one 16-byte store per
-  // thread when the tile is exactly one group of one page
-  const int d = tid;
-  float xv[kTok];
+  // ---- V: thread (q, c) = (tid / (D/4), tid % (D/4)) loads head dims
+  // 4c .. 4c + 3 of the four tokens 2q, 2q + 1, 2q + 8, 2q + 9 (one 16-byte
+  // load per token for f32, 8 bytes for bf16): exactly the four slots that
+  // share word q of a 16-slot group row, so each of its four dims yields one
+  // 32-bit word.  The words meet in shared memory ([d][16 slots], the group
+  // row layout) and thread d stores its dimension's row -- one 16-byte write
+  // when the 16 tokens fill one group of one page (the cache-fill case),
+  // single bytes otherwise (a decode step's few tokens).
+  constexpr int C4 = D / 4;
+  const int vq = tid / C4, vc = tid % C4;
+  int vt[4];
+  vt[0] = 2 * vq;
+  vt[1] = 2 * vq + 1;
+  vt[2] = 2 * vq + 8;
+  vt[3] = 2 * vq + 9;
+  float xv[4][4];  // [token k of the four][dim e]
 #pragma unroll
-  for (int t = 0; t < kTok; ++t) {
-    xv[t] = 0.f;
+  for (int k = 0; k < 4; ++k) {
+    const int t = vt[k];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) xv[k][e] = 0.f;
     if (t < n_tok) {
-      const size_t e = (((size_t)b * p.n_new + t0 + t) * p.Hkv + h) * D + d;
-      xv[t] = (p.dtype == ATLAS_DTYPE_F32)
-                  ? __ldg(static_cast<const float*>(p.v_new) + e)
-                  : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p.v_new) + e));
+      const size_t el = (((size_t)b * p.n_new + t0 + t) * p.Hkv + h) * D + 4 * vc;
+      if (p.dtype == ATLAS_DTYPE_F32) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(p.v_new) + el));
+        xv[k][0] = f.x; xv[k][1] = f.y; xv[k][2] = f.z; xv[k][3] = f.w;
+      } else {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(
+            static_cast<const __nv_bfloat16*>(p.v_new) + el));
+        xv[k][0] = __uint_as_float(w.x << 16); xv[k][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        xv[k][2] = __uint_as_float(w.y << 16); xv[k][3] = __uint_as_float(w.y & 0xFFFF0000u);
+      }
     }
   }
-  float vsc[kTok];
-  if constexpr (TS) {  // per-token scales: the row maximum over all D threads
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      float a = fabsf(xv[t]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-      if ((tid & 31) == 0) s_amax[tid >> 5][t] = a;
-    }
-  }
-  __syncthreads();  // s_page (and s_amax) ready
+  float vsc[4];  // the four tokens' V scales
   if constexpr (TS) {
+    // per-token scales: the token's row maximum over all D dims -- the C4
+    // threads of one q hold the row (one warp at D = 128, half a warp at 64)
 #pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      float a = s_amax[0][t];
+    for (int k = 0; k < 4; ++k) {
+      float a = fmaxf(fmaxf(fabsf(xv[k][0]), fabsf(xv[k][1])), fmaxf(fabsf(xv[k][2]), fabsf(xv[k][3])));
 #pragma unroll
-      for (int w = 1; w < NW; ++w) a = fmaxf(a, s_amax[w][t]);
-      vsc[t] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+      for (int o = C4 / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      vsc[k] = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
     }
   } else {
     const float s0 = __ldg(p.v_scale + h);
 #pragma unroll
-    for (int t = 0; t < kTok; ++t) vsc[t] = s0;
+    for (int k = 0; k < 4; ++k) vsc[k] = s0;
   }
-  uint32_t code[kTok];
+  __shared__ __align__(16) uint32_t s_v[D][4];  // [d][word]: group row of dim d
 #pragma unroll
-  for (int t = 0; t < kTok; t += 2) {
-    const float y0 = __fdiv_rn(xv[t], vsc[t]), y1 = __fdiv_rn(xv[t + 1], vsc[t + 1]);
-    const uint32_t pr = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
-    code[t] = pr & 0xFFu;
-    code[t + 1] = (pr >> 8) & 0xFFu;
+  for (int e = 0; e < 4; ++e) {
+    // word q of dim 4c + e: bytes = slots 2q, 2q + 1, 2q + 8, 2q + 9
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(xv[0][e], vsc[0]), __fdiv_rn(xv[1][e], vsc[1])), __NV_SATFINITE,
+        __NV_E4M3);
+    const uint32_t hi2 = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(xv[2][e], vsc[2]), __fdiv_rn(xv[3][e], vsc[3])), __NV_SATFINITE,
+        __NV_E4M3);
+    s_v[4 * vc + e][vq] = (lo & 0xFFFFu) | ((hi2 & 0xFFFFu) << 16);
+  }
+  __syncthreads();  // the group rows (and s_page) are complete
+  if (TS && vc == 0) {  // the four tokens' V scales and the head's bound
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = vt[k];
+      if (t >= n_tok || s_page[t] < 0) continue;
+      const int slot = (start + t0 + t) % p.ps;
+      p.v_tok_scale[((size_t)s_page[t] * p.Hkv + h) * p.ps + slot] = vsc[k];
+      // positive floats order like their bit patterns: the head's running
+      // bound of the per-token V scales
+      atomicMax(reinterpret_cast<int*>(p.v_scale_bound + h), __float_as_int(vsc[k]));
+    }
   }
   const int p0 = start + t0;
   const bool whole_group = n_tok == kTok && (p0 % 16) == 0 && s_page[0] >= 0;
-  if (whole_group) {
-    // slot t of the group sits at byte 4*((t%8)/2) + 2*(t/8) + t%2: word c
-    // holds slots 2c, 2c+1, 2c+8, 2c+9
-    uint32_t w[4];
+  {
+    const int d = tid;  // this thread's dimension: its 16 codes in group order
+    const uint4 row = *reinterpret_cast<const uint4*>(&s_v[d][0]);
+    if (whole_group) {
+      const size_t head_page = (size_t)s_page[0] * p.Hkv + h;
+      uint8_t* dst = p.v_pages + (head_page * (p.ps / 16) + (p0 % p.ps) / 16) * (16 * D) + 16 * d;
+      *reinterpret_cast<uint4*>(dst) = row;
+    } else {  // byte stores for the valid tokens (a decode step's few tokens)
+      const uint32_t rw[4] = {row.x, row.y, row.z, row.w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      w[c] = code[2 * c] | (code[2 * c + 1] << 8) | (code[2 * c + 8] << 16) |
-             (code[2 * c + 9] << 24);
-    const size_t head_page = (size_t)s_page[0] * p.Hkv + h;
-    uint8_t* dst = p.v_pages + (head_page * (p.ps / 16) + (p0 % p.ps) / 16) * (16 * D) + 16 * d;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {  // byte stores for the valid tokens (a decode step's few tokens)
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      const int pg = s_page[t];
-      if (t >= n_tok || pg < 0) continue;
-      const int slot = (p0 + t) % p.ps;
-      const int g = slot % 16;
-      const int byte = 4 * ((g & 7) >> 1) + 2 * (g >> 3) + (g & 1);
-      const size_t head_page = (size_t)pg * p.Hkv + h;
-      p.v_pages[(head_page * (p.ps / 16) + slot / 16) * (16 * D) + 16 * d + byte] =
-          (uint8_t)code[t];
+      for (int t = 0; t < kTok; ++t) {
+        const int pg = s_page[t];
+        if (t >= n_tok || pg < 0) continue;
+        const int slot = (p0 + t) % p.ps;
+        const int g = slot % 16;
+        const int byte = 4 * ((g & 7) >> 1) + 2 * (g >> 3) + (g & 1);
+        const int tb = 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);  // token t in the row
+        const size_t head_page = (size_t)pg * p.Hkv + h;
+        p.v_pages[(head_page * (p.ps / 16) + slot / 16) * (16 * D) + 16 * d + byte] =
+            (uint8_t)(rw[tb >> 2] >> (8 * (tb & 3)));
+      }
     }
-  }
-  if (TS && d < n_tok && s_page[d] >= 0) {  // thread t < 16 stores token t's V scale
-    float a = s_amax[0][d];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) a = fmaxf(a, s_amax[w][d]);
-    const float sc = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-    const int slot = (p0 + d) % p.ps;
-    p.v_tok_scale[((size_t)s_page[d] * p.Hkv + h) * p.ps + slot] = sc;
-    // positive floats order like their bit patterns: the head's running bound
-    // of the per-token V scales
-    atomicMax(reinterpret_cast<int*>(p.v_scale_bound + h), __float_as_int(sc));
   }
 
   // ---- K, 16 consecutive elements of one token row per thread (one
