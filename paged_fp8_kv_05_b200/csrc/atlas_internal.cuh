@@ -315,6 +315,124 @@ void decode_fp8_fit_grid(int D, int rows, int sms, DecodeLaunch& L);
 
 #ifdef __CUDACC__
 
+// A1, the order of the grid partition's work.  Its items are (sequence b,
+// segment, split): a served sequence of length L has n = ceil(L / T) splits,
+// and Hs segments (KV head x row block) each.  The items are ranked by a
+// length key, largest first: every split of a sequence cut in n >= 2 splits
+// counts as a whole split (ceil(T / 128) tiles), so that these sequences
+// come first, segment-major (the splits of a segment neighbours: they end
+// together and the segment's merge of its partials is not left for the end
+// of the launch); a sequence served by one split ranks by its own number of
+// 128-token tiles, so the shortest come last and fill the end of the launch.
+// Ties by sequence.  Ranks past the last item (splits past a sequence's end)
+// come last.  Every thread of the CTA calls it (it synchronises the CTA); it
+// returns false when rank `ci` is past the last item, else the item.
+// `served(bb, L)` says whether sequence bb of length L is served.  Shared
+// memory: hist ceil(T / 128) + 1 ints, wsum one int per warp, res 4 ints.
+template <int NTHREADS, class Served>
+__device__ __forceinline__ bool longest_first_item(long long ci, int B,
+                                                   const int32_t* __restrict__ seq_lens, int T,
+                                                   int Hs, Served served, int* hist, int* wsum,
+                                                   int* res, int& b, int& seg, int& split) {
+  constexpr int NW = NTHREADS / 32;
+  constexpr unsigned kAll = 0xFFFFFFFFu;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int TT = (T + 127) / 128;  // tiles of a whole split: the top key
+  auto key_of = [&](int L, int n) { return n >= 2 ? TT : (L + 127) / 128; };
+  for (int i = tid; i <= TT; i += NTHREADS) hist[i] = 0;
+  __syncthreads();
+  // sequences per key (each holds n x Hs items)
+  long long top = 0;  // items of key TT
+  for (int bb = tid; bb < B; bb += NTHREADS) {
+    const int L = __ldg(seq_lens + bb);
+    if (!served(bb, L)) continue;
+    const int n = (L + T - 1) / T;
+    const int k = key_of(L, n);
+    if (k == TT)
+      top += n;
+    else
+      atomicAdd(&hist[k], 1);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) top += __shfl_xor_sync(kAll, top, o);
+  if (lane == 0 && top > 0) atomicAdd(&hist[TT], (int)top);
+  __syncthreads();
+  // warp 0: the key (bin) of item rank ci and its rank within the bin,
+  // scanning the bins from TT down, 32 at a time (bin counts in items)
+  if (warp == 0) {
+    long long base = 0, rank = 0;
+    int bin = -1;
+    for (int t0 = TT; t0 >= 1; t0 -= 32) {
+      const int k = t0 - lane;
+      const long long c = k >= 1 ? (long long)hist[k] * Hs : 0;
+      long long incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long u = __shfl_up_sync(kAll, incl, o);
+        if (lane >= o) incl += u;
+      }
+      const long long excl = base + incl - c;
+      const unsigned hit = __ballot_sync(kAll, c > 0 && ci >= excl && ci < excl + c);
+      if (bin < 0 && hit) {
+        const int src = __ffs(hit) - 1;
+        bin = __shfl_sync(kAll, k, src);
+        rank = ci - __shfl_sync(kAll, excl, src);
+      }
+      base += __shfl_sync(kAll, incl, 31);
+    }
+    if (lane == 0) {
+      res[0] = bin;
+      res[1] = (int)rank;  // < B * n * Hs: the grid size, an int
+      res[2] = -1;
+    }
+  }
+  __syncthreads();
+  const int bin = res[0], rank = res[1];
+  if (bin < 0) return false;  // CTA-uniform
+  // the rank-th item of the bin, in sequence order: sequence bb holds n x Hs
+  // items of its key, segment-major
+  long long done = 0;
+  for (int b0 = 0; b0 < B && done <= rank; b0 += NTHREADS) {
+    const int bb = b0 + tid;
+    int c = 0, n = 0;
+    if (bb < B) {
+      const int L = __ldg(seq_lens + bb);
+      if (served(bb, L)) {
+        n = (L + T - 1) / T;
+        c = key_of(L, n) == bin ? n : 0;
+      }
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(kAll, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int x = wsum[w];
+      before += w < warp ? x : 0;
+      total += x;
+    }
+    // index among this sequence's items
+    const long long j = rank - (done + (long long)(before + incl - c) * Hs);
+    if (c > 0 && j >= 0 && j < (long long)c * Hs) {
+      res[2] = bb;
+      res[3] = (int)(j / n);  // segment
+      res[0] = (int)(j % n);  // split
+    }
+    done += (long long)total * Hs;
+    __syncthreads();  // wsum free for the next chunk; res written
+  }
+  b = res[2];
+  seg = res[3];
+  split = res[0];
+  return b >= 0;  // both passes count the same items, so b >= 0 here
+}
+
 // f16x2 with `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;

@@ -14,7 +14,12 @@
 //
 // CTA = one split of one segment (sequence b, KV head h, block of up to 64
 // query rows), as in the grid partition: split_tokens KV tokens in tiles of
-// 128.  Six warps:
+// 128.  The CTAs take their items longest first: every CTA ranks the items
+// by a length key from seq_lens (a histogram and two block scans) and takes
+// the one its index names -- the sequences cut into several splits first,
+// segment-major, then the single-split ones by their number of tiles, so the
+// short ones fill the end of the launch and the indices past the last item
+// (splits past a sequence's end) come last.  Six warps:
 //   * warp 4 -- producer: 1-D bulk copies (cp.async.bulk, no multicast) of
 //     the tile's eight 16-token K pieces and eight V pieces (pieces adjacent
 //     in a page go as one copy, one lane per run) into a K ring and a V ring
@@ -70,6 +75,8 @@ constexpr uint32_t kColS = 0;              // S double buffer: columns 0-63, 64-
 constexpr uint32_t kColO = 128;            // O: columns 128-191
 constexpr uint32_t kColQ = 192;            // Q hi: 192-223, Q lo: 224-255 (A operand)
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSchedExtra = kWarps + 4;    // scan partials + (bin, rank, b, split)
 
 // ---------------------------------------------------------------- tcgen05 PTX
 
@@ -275,7 +282,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // ----------------------------------------------------------- shared memory
 
 struct TcLayout {
-  size_t k, v, ts, p, tab, bar, misc, rows, total;
+  size_t k, v, ts, p, tab, sched, bar, misc, rows, total;
 };
 // E4M3 parts that carry a probability into the PV product: hi + lo (8
 // significant bits); three with per-token V scales, where even the row's
@@ -293,7 +300,9 @@ __host__ __device__ inline TcLayout tc_layout(int k_stages, int max_pieces, bool
   t.ts = t.v + (size_t)kVS * kTileBytes;                // [KS][128] K scales, [kVS][128] V scales
   t.p = t.ts + (tok_scales ? (size_t)(k_stages + kVS) * kTile * 4 : 0);  // P parts: core matrices
   t.tab = t.p + (size_t)p_parts(tok_scales) * kOpBytes; // piece table, int32 per 16 tokens
-  t.bar = (t.tab + (size_t)max_pieces * 4 + 15) / 16 * 16;
+  t.sched = t.tab + (size_t)max_pieces * 4;             // work order: pairs per tile count
+                                                        // [tiles + 1], scan partials, result
+  t.bar = (t.sched + (size_t)(max_pieces / 8 + 1 + kSchedExtra) * 4 + 15) / 16 * 16;
   t.misc = t.bar + (size_t)tc_barriers(k_stages) * 8;   // tmem address, abort flag, is_last
   t.rows = t.k;                                         // merge: row reference, denominator
                                                         // (after the tiles: K stage 0)
@@ -362,15 +371,28 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_tc_kernel(const Deco
     for (size_t idx = tid; idx < n; idx += kThreads) o[idx] = __float2bfloat16_rn(0.f);
   }
 
+  // ---- A1, the work order: this CTA's item (sequence, segment, split),
+  // longest first
+  const int T = p.split_tokens;
+  int b, seg, split;
+  {
+    int* hist = reinterpret_cast<int*>(smem + lay.sched);  // [T / 128 + 1]
+    int* wsum = hist + T / kTile + 1;                       // [kWarps]
+    int* res = wsum + kWarps;                               // [4]
+    auto served = [&](int bb, int Lb) { return valid_len(Lb, qlen_of(bb)); };
+    if (!longest_first_item<kThreads>(cid, p.B, p.seq_lens, T, Hs, served, hist, wsum, res, b,
+                                      seg, split))
+      return;  // past the last item (CTA-uniform)
+  }
+
   // ---- this CTA's split (A1): tokens [t_begin, t_end) of segment (b, h, rb)
-  const int split = cid % p.num_splits, sg = cid / p.num_splits;
-  const int b = sg / Hs, seg = sg % Hs, h = seg / RB, rb = seg % RB;
+  const int sg = b * Hs + seg;
+  const int h = seg / RB, rb = seg % RB;
   const int L = __ldg(p.seq_lens + b);
   const int q_len = qlen_of(b), q_base = qbase_of(b);
   if (!valid_len(L, q_len)) return;        // CTA-uniform; rows zeroed above
   const int Rtot = q_len * p.G;            // this sequence's query rows per KV head
   if (rb * kRows >= Rtot) return;          // a row block past this sequence's rows
-  const int T = p.split_tokens;
   const int t_begin = split * T;
   if (t_begin >= L) return;
   const int t_end = min(L, t_begin + T);
