@@ -199,3 +199,37 @@ def test_tc_lost_copy_times_out_and_the_library_stays_usable(ak):
     again = dw.decode(out=torch.empty_like(dw.q))
     assert dw.pool.device_error() == 0
     assert_close(again.float().cpu().numpy(), ref, "the call after the timeout")
+
+
+def test_tc_work_order_serves_every_item_once(ak):
+    """The CTAs rank their (sequence, segment, split) items in-kernel, longest
+    first.  230 sequences (more than one 192-sequence chunk of the rank
+    search) with lengths on every side of the 128-token tile and 256-token
+    split boundaries, and three sequences the kernel must skip (length 0 <
+    q_len) spread over both chunks: every served row matches the oracle (no
+    item lost: the output starts as NaN; none served twice: the split partials
+    would not merge to the oracle), the skipped ones are zero and flagged."""
+    base = [1, 2, 127, 128, 129, 200, 255, 256, 257, 300, 383, 384, 385, 511, 512,
+            513, 640, 700, 767, 768, 769, 1000, 1023, 1024, 1025]
+    rng = np.random.default_rng(5)
+    lens = [int(x) for x in rng.permutation(np.resize(base, 230))]
+    w = _case(230, 8, 2, 128, 16, lens, 1, seed=23)
+    dw = _dw(w)
+    dw.pool.set_option(ak.OPT_KERNEL, ak.KERNEL_TC)
+    dw.pool.set_split_tokens(256)
+    plan = dw.plan()
+    assert plan["kernel"] == 3 and plan["split_tokens"] == 256
+    skip = [0, 150, 229]
+    sl = dw.seq_lens.clone()
+    sl[skip] = 0
+    out = torch.full_like(dw.q, float("nan"))
+    ak.atlas_paged_gqa_decode(dw.pool, dw.q, dw.block_table, sl, w.max_seq_len, out=out)
+    err = dw.pool.device_error()
+    assert err & ak.DEVERR_SEQ_LEN and not err & ~ak.DEVERR_SEQ_LEN, err
+    got = out.float().cpu().numpy()
+    assert np.all(got[skip] == 0)
+    keep = np.ones(len(lens), bool)
+    keep[skip] = False
+    ref = oracle_decode(w)
+    max_abs, rel = assert_close(got[keep], ref[keep], "tcgen05 work order, 230 sequences")
+    record_parity("tcgen05 work order, 230 sequences, split 256", max_abs, rel)
