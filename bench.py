@@ -579,6 +579,30 @@ def accept_throughput(device, flush_l2, ak, batch=128, num_drafts=4, vocab=15193
             "launches_per_call": 1}
 
 
+def stage_inputs(parts, pin=False):
+    """Pack tensors into one uint8 buffer, each at a 256-byte-aligned offset
+    (the end-to-end leg's single host-to-device copy).  Returns the buffer
+    (pinned if asked) and the offsets."""
+    offs, n = [], 0
+    for t in parts:
+        offs.append(n)
+        n = (n + t.numel() * t.element_size() + 255) // 256 * 256
+    buf = torch.zeros(n, dtype=torch.uint8)
+    if pin:
+        buf = buf.pin_memory()
+    for t, o in zip(parts, offs):
+        nb = t.numel() * t.element_size()
+        buf[o:o + nb].copy_(t.contiguous().reshape(-1).view(torch.uint8))
+    return buf, offs
+
+
+def staged_views(buf, parts, offs):
+    """Views into a staging buffer (or its device copy) with the dtypes and
+    shapes of `parts`."""
+    return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+            for t, o in zip(parts, offs)]
+
+
 def measure(index, args, device, dist, ak, flush_l2, local):
     """Time K fused steps (append + decode, one launch each) of one workload,
     then K_e2e steps end to end through the public API with pinned host
@@ -640,21 +664,12 @@ def measure(index, args, device, dist, ak, flush_l2, local):
              torch.from_numpy(w.new_tokens("v")),
              torch.from_numpy(w.seq_lens.astype(np.int32)),
              torch.from_numpy(np.ascontiguousarray(w.block_table))]
-    offs, n = [], 0
-    for t in parts:
-        offs.append(n)
-        n = (n + t.numel() * t.element_size() + 255) // 256 * 256
-    stage_h = torch.zeros(n, dtype=torch.uint8).pin_memory()
-    for t, o in zip(parts, offs):
-        nb = t.numel() * t.element_size()
-        stage_h[o:o + nb].copy_(t.reshape(-1).view(torch.uint8))
-    stage_d = torch.empty(n, dtype=torch.uint8, device=device)
-    q_d, k_d, v_d, sl_d, bt_d = (
-        stage_d[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
-        for t, o in zip(parts, offs))
+    stage_h, offs = stage_inputs(parts, pin=True)
+    stage_d = torch.empty(stage_h.numel(), dtype=torch.uint8, device=device)
+    q_d, k_d, v_d, sl_d, bt_d = staged_views(stage_d, parts, offs)
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
     out_d = torch.empty_like(dw.q)
-    h2d = n
+    h2d = stage_h.numel()
     d2h = out_h.numel() * out_h.element_size()
     K_e2e = min(K, 200)
     e2e_ms = []
