@@ -301,8 +301,10 @@ ATLAS_API atlas_status_t atlas_paged_gqa_decode_tokscale(
  * and flags ATLAS_DEVERR_PAGE_ID.  batch == 0 is a no-op.  Uses the pool workspace.
  * Partition (ATLAS_OPT_PARTITION): each (sequence, KV head, row block)
  * segment is cut into splits of a fixed number of tokens, one CTA each, that
- * the hardware hands to SMs as they free up; or the 32-token units of all
- * segments are cut into equal ranges, one per CTA, whatever the length mix.
+ * the hardware hands to SMs as they free up (the tensor-core kernel's CTAs
+ * take these splits longest first, ranked in the kernel from seq_lens); or
+ * the 32-token units of all segments are cut into equal ranges, one per CTA,
+ * whatever the length mix.
  * A segment cut in several parts is merged by log-sum-exp by the CTA that
  * finishes it last.  A wait that runs out (200 ms) flags ATLAS_DEVERR_TIMEOUT.
  */
